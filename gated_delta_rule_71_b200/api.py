@@ -1,0 +1,178 @@
+"""Thin PyTorch-facing binding of libgdn.so.
+
+PyTorch supplies device memory and the current CUDA stream; every step of the
+computation runs in the library's kernels.  Each function checks shapes,
+dtypes and devices, allocates outputs with torch, and forwards raw pointers.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+F32, BF16 = 0, 1
+FLAG_EXACT_F32 = 0x1
+FLAG_CHUNK32 = 0x10
+FLAG_CHUNK16 = 0x20
+FLAG_VSPLIT1 = 0x100
+FLAG_VSPLIT2 = 0x200
+FLAG_VSPLIT4 = 0x400
+
+_DT = {torch.float32: F32, torch.bfloat16: BF16}
+
+
+def _stream(t: torch.Tensor):
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, device=None, contiguous=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gate_prep(a: torch.Tensor, b: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor,
+              beta: Optional[torch.Tensor] = None, g: Optional[torch.Tensor] = None
+              ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """beta = sigmoid(b), g = -exp(A_log) * softplus(a + dt_bias); a, b [..., H] fp32."""
+    H = a.shape[-1]
+    dev = a.device
+    for t, n in ((a, "a"), (b, "b")):
+        _need(t, n, torch.float32, dev, contiguous=False)
+    a2 = a.reshape(-1, H)
+    b2 = b.reshape(-1, H)
+    if a2.stride(-1) != 1 or b2.stride(-1) != 1:
+        raise ValueError("a and b need a contiguous head dimension")
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias")):
+        _need(t, n, torch.float32, dev)
+    beta = torch.empty(a.shape, dtype=torch.float32, device=dev) if beta is None else beta
+    g = torch.empty(a.shape, dtype=torch.float32, device=dev) if g is None else g
+    _need(beta, "beta", torch.float32, dev)
+    _need(g, "g", torch.float32, dev)
+    _lib.call("gdn_gate_prep", _ptr(a2), _ptr(b2), a2.shape[0], H, a2.stride(0), b2.stride(0),
+              _ptr(A_log), _ptr(dt_bias), _ptr(beta), _ptr(g), _stream(a))
+    return beta, g
+
+
+def chunk_fwd_workspace_size(n_seq: int, T_total: int, H: int, K: int, V: int,
+                             dtype=torch.bfloat16) -> int:
+    return int(_lib.load().gdn_chunk_fwd_workspace_size(n_seq, T_total, H, K, V, _DT[dtype]))
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+              beta: torch.Tensor, h0: Optional[torch.Tensor] = None,
+              cu_seqlens: Optional[torch.Tensor] = None, scale: float = 1.0,
+              o_dtype: torch.dtype = torch.float32, output_final_state: bool = True,
+              flags: int = 0, workspace: Optional[torch.Tensor] = None,
+              out: Optional[torch.Tensor] = None, hT: Optional[torch.Tensor] = None
+              ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked gated delta rule.  q, k [B,T,H,K]; v [B,T,H,V]; g, beta [B,T,H] fp32;
+    h0 [n_seq,H,K,V] fp32 or None; cu_seqlens int32 [n_seq+1] (B == 1) or None.
+    Returns (o [B,T,H,V] in o_dtype, hT [n_seq,H,K,V] fp32 or None)."""
+    dev = q.device
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype: float32 or bfloat16")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    if tuple(k.shape) != (B, T, H, K) or tuple(v.shape[:3]) != (B, T, H):
+        raise ValueError("shape mismatch among q, k, v")
+    for t, n in ((g, "g"), (beta, "beta")):
+        _need(t, n, torch.float32, dev)
+        if tuple(t.shape) != (B, T, H):
+            raise ValueError(f"{n} must be [B, T, H]")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if B != 1:
+            raise ValueError("packed sequences need B == 1")
+        n_seq = cu_seqlens.numel() - 1
+    else:
+        n_seq = B
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, dev)
+        if tuple(h0.shape) != (n_seq, H, K, V):
+            raise ValueError("h0 must be [n_seq, H, K, V]")
+    if out is None:
+        out = torch.empty((B, T, H, V), dtype=o_dtype, device=dev)
+    _need(out, "out", o_dtype, dev)
+    if output_final_state and hT is None:
+        hT = torch.empty((n_seq, H, K, V), dtype=torch.float32, device=dev)
+    if hT is not None:
+        _need(hT, "hT", torch.float32, dev)
+    ws_need = chunk_fwd_workspace_size(n_seq, B * T, H, K, V, q.dtype)
+    if ws_need and workspace is None:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    _lib.call("gdn_chunk_fwd", _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(g), _ptr(beta),
+              _ptr(h0), _ptr(cu_seqlens), n_seq, B, T, H, K, V, float(scale), _ptr(out),
+              _DT[o_dtype], _ptr(hT), _ptr(workspace),
+              0 if workspace is None else workspace.numel() * workspace.element_size(),
+              int(flags), _stream(q))
+    return out, hT
+
+
+def _decode_common(x, ba, A_log, dt_bias, M, H, G, P, N):
+    dev = x.device
+    _need(x, "x", torch.bfloat16, dev, contiguous=False)
+    _need(ba, "ba", torch.bfloat16, dev, contiguous=False)
+    if x.stride(-1) != 1 or ba.stride(-1) != 1:
+        raise ValueError("x and ba need a contiguous last dimension")
+    n = x.shape[0]
+    width = M * H * P + M * G * N + G * N
+    if x.shape[-1] != width or ba.shape[-1] != M * H + H:
+        raise ValueError("x / ba last dimension does not match M, H, G, P, N")
+    for t, nm in ((A_log, "A_log"), (dt_bias, "dt_bias")):
+        _need(t, nm, torch.float32, dev)
+    return dev, n, x.stride(0), ba.stride(0)
+
+
+def gdp_decode_prepare(x, ba, A_log, dt_bias, M, H, G, P, N):
+    """Returns q, k [n,M,H,N] bf16, v [n,M,H,P] bf16, beta, g [n,M,H] fp32."""
+    dev, n, xs, bas = _decode_common(x, ba, A_log, dt_bias, M, H, G, P, N)
+    q = torch.empty((n, M, H, N), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((n, M, H, N), dtype=torch.bfloat16, device=dev)
+    v = torch.empty((n, M, H, P), dtype=torch.bfloat16, device=dev)
+    beta = torch.empty((n, M, H), dtype=torch.float32, device=dev)
+    g = torch.empty((n, M, H), dtype=torch.float32, device=dev)
+    _lib.call("gdp_decode_prepare", _ptr(x), xs, _ptr(ba), bas, _ptr(A_log), _ptr(dt_bias), n, M,
+              H, G, P, N, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _stream(x))
+    return q, k, v, beta, g
+
+
+def gdp_decode_step(x, ba, A_log, dt_bias, state, M, H, G, P, N, scale=1.0, qk_l2norm=True,
+                    out=None):
+    """Fused decode step; updates state [n,H,N,P] fp32 in place, returns o [n,H,P] bf16."""
+    dev, n, xs, bas = _decode_common(x, ba, A_log, dt_bias, M, H, G, P, N)
+    _need(state, "state", torch.float32, dev)
+    if tuple(state.shape) != (n, H, N, P):
+        raise ValueError("state must be [n, H, N, P]")
+    if out is None:
+        out = torch.empty((n, H, P), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _lib.call("gdp_decode_step", _ptr(x), xs, _ptr(ba), bas, _ptr(A_log), _ptr(dt_bias), n, M, H,
+              G, P, N, _ptr(state), _ptr(out), float(scale), int(bool(qk_l2norm)), _stream(x))
+    return out
+
+
+def device_status(device=None) -> int:
+    """Reads and clears the device status word (synchronises the current stream)."""
+    s = torch.cuda.current_stream(device).cuda_stream
+    return int(_lib.load().gdn_device_status(s))
+
+
+def selftest_wait_timeout(polls: int = 64, device=None) -> None:
+    s = torch.cuda.current_stream(device).cuda_stream
+    _lib.call("gdn_selftest_wait_timeout", int(polls), s)

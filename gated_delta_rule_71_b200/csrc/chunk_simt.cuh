@@ -1,0 +1,247 @@
+// chunk_simt.cuh -- fp32-FMA chunked forward of the gated delta rule, and the
+// packed-batch schedule map.
+//
+// Chunked form (64-token chunks by default; C = 16 / 32 for invariance tests),
+// derived from the rule S_t = exp(g_t) S_{t-1}(I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+// with h = S^T.  For one chunk with in-chunk inclusive cumsum G_r of g, state h
+// at chunk start and r, s in [0, C):
+//   A    = strictly-lower [ beta_r exp(G_r - G_s) k_r . k_s ]          (C x C)
+//   T    = (I + A)^-1                     (forward substitution)
+//   R    = diag(beta) (V - diag(exp(G)) K h)
+//   Ut   = T R                            ( = U - W h with W = T diag(beta e^G) K,
+//                                             U = T diag(beta) V )
+//   O    = scale [ diag(exp(G)) Q h + (lower-incl [ exp(G_r - G_s) q_r . k_s ]) Ut ]
+//   h'   = exp(G_L) h + (diag(exp(G_L - G_r)) K)^T Ut
+// ZzCompute (PyTorch Helion Hackathon gallery entry 11): item 4 "Recompute W/U"
+// (WY transform), item 2 "Chunk Forward H" (state recurrence: delta
+// correction, decay gating, accumulation), item 3 "Chunk Forward O" (state
+// query plus intra-chunk causal attention).  Every product here stays in IEEE
+// fp32, the precision item 2 asks for.
+//
+// One block per (sequence, head, V-slice); the V columns never interact, so
+// slices run their recurrences independently.  Tail rows of a chunk get
+// beta = g = 0 and zero q/k/v, which makes them exact identities.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdn {
+
+struct ChunkArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* h0;
+    const int32_t* cu_seqlens;  // NULL: dense
+    const int32_t* order;       // NULL: identity schedule
+    int n_seq;
+    int64_t T;  // dense sequence length
+    int H, K, V;
+    int VS;  // V-slice width
+    int nvs; // number of V-slices
+    float scale;
+    void* o;
+    float* hT;
+};
+
+__device__ __forceinline__ void seq_bounds(const ChunkArgs& a, int seq, int64_t& cs, int64_t& ce) {
+    if (a.cu_seqlens) {
+        cs = a.cu_seqlens[seq];
+        ce = a.cu_seqlens[seq + 1];
+    } else {
+        cs = (int64_t)seq * a.T;
+        ce = cs + a.T;
+    }
+}
+
+// Floats of shared memory the fp32 kernel needs for chunk C, key dim K and
+// V-slice VS.
+__host__ __device__ constexpr int64_t simt_smem_floats(int C, int K, int VS) {
+    return 2LL * C * (K + 1) + 3LL * C * VS + (int64_t)K * VS + 2LL * C * (C + 1) + 4LL * C;
+}
+
+template <int C, typename TIn, typename TOut>
+__global__ void __launch_bounds__(256) chunk_fwd_simt_kernel(ChunkArgs a) {
+    extern __shared__ float smem[];
+    const int K = a.K, V = a.V, VS = a.VS, H = a.H;
+    const int KP = K + 1, CP = C + 1;
+    float* sK = smem;              // [C][K+1]
+    float* sQ = sK + C * KP;       // [C][K+1]
+    float* sR = sQ + C * KP;       // [C][VS]  v slice, then R
+    float* sQH = sR + C * VS;      // [C][VS]  exp(G) Q h
+    float* sU = sQH + C * VS;      // [C][VS]  Ut
+    float* sH = sU + C * VS;       // [K][VS]  state slice
+    float* sA = sH + K * VS;       // [C][C+1] A, then T
+    float* sP = sA + C * CP;       // [C][C+1] causal decayed Q K^T
+    float* sG = sP + C * CP;       // [C] cumsum of g
+    float* sB = sG + C;            // [C] beta
+    float* sGam = sB + C;          // [C] exp(G_r)
+    float* sW = sGam + C;          // [C] exp(G_L - G_r)
+
+    const int tid = threadIdx.x, nth = blockDim.x;
+    const int vsl = blockIdx.x % a.nvs;
+    const int sh = blockIdx.x / a.nvs;
+    const int head = sh % H;
+    const int slot = sh / H;
+    const int seq = a.order ? a.order[slot] : slot;
+    const int v0 = vsl * VS;
+    int64_t cs, ce;
+    seq_bounds(a, seq, cs, ce);
+
+    const TIn* q = static_cast<const TIn*>(a.q);
+    const TIn* k = static_cast<const TIn*>(a.k);
+    const TIn* v = static_cast<const TIn*>(a.v);
+    TOut* o = static_cast<TOut*>(a.o);
+
+    // initial state slice
+    const int64_t hbase = ((int64_t)seq * H + head) * K * V;
+    for (int i = tid; i < K * VS; i += nth) {
+        const int c = i / VS, j = i - c * VS;
+        sH[i] = a.h0 ? a.h0[hbase + (int64_t)c * V + v0 + j] : 0.f;
+    }
+
+    for (int64_t t0 = cs; t0 < ce; t0 += C) {
+        const int len = (int)min((int64_t)C, ce - t0);
+        __syncthreads();  // previous chunk fully consumed
+        // ---- load chunk (tail rows -> zeros, beta = g = 0)
+        for (int i = tid; i < C * K; i += nth) {
+            const int r = i / K, c = i - r * K;
+            float kk = 0.f, qq = 0.f;
+            if (r < len) {
+                const int64_t row = ((t0 + r) * H + head) * (int64_t)K;
+                kk = to_f32(k[row + c]);
+                qq = to_f32(q[row + c]);
+            }
+            sK[r * KP + c] = kk;
+            sQ[r * KP + c] = qq;
+        }
+        for (int i = tid; i < C * VS; i += nth) {
+            const int r = i / VS, j = i - r * VS;
+            sR[i] = (r < len) ? to_f32(v[((t0 + r) * H + head) * (int64_t)V + v0 + j]) : 0.f;
+        }
+        for (int r = tid; r < C; r += nth) {
+            const bool ok = r < len;
+            sG[r] = ok ? a.g[(t0 + r) * H + head] : 0.f;
+            sB[r] = ok ? a.beta[(t0 + r) * H + head] : 0.f;
+        }
+        __syncthreads();
+        // ---- in-chunk cumsum of g and the decay factors
+        if (tid == 0) {
+            float acc = 0.f;
+            for (int r = 0; r < C; ++r) {
+                acc += sG[r];
+                sG[r] = acc;
+            }
+        }
+        __syncthreads();
+        const float GL = sG[C - 1];
+        for (int r = tid; r < C; r += nth) {
+            sGam[r] = expf(sG[r]);
+            sW[r] = expf(GL - sG[r]);
+        }
+        // ---- A, causal P, and the state products K h, Q h
+        for (int i = tid; i < C * C; i += nth) {
+            const int r = i / C, s = i - r * C;
+            float av = 0.f, pv = 0.f;
+            if (s <= r) {
+                float dk = 0.f, dq = 0.f;
+                for (int c = 0; c < K; ++c) {
+                    const float ks = sK[s * KP + c];
+                    dk = fmaf(sK[r * KP + c], ks, dk);
+                    dq = fmaf(sQ[r * KP + c], ks, dq);
+                }
+                const float d = expf(sG[r] - sG[s]);
+                pv = d * dq;
+                if (s < r) av = sB[r] * d * dk;
+            }
+            sA[r * CP + s] = av;
+            sP[r * CP + s] = pv;
+        }
+        for (int i = tid; i < C * VS; i += nth) {
+            const int r = i / VS, j = i - r * VS;
+            float kh = 0.f, qh = 0.f;
+            for (int c = 0; c < K; ++c) {
+                const float hv = sH[c * VS + j];
+                kh = fmaf(sK[r * KP + c], hv, kh);
+                qh = fmaf(sQ[r * KP + c], hv, qh);
+            }
+            const float gam = expf(sG[r]);
+            sR[i] = sB[r] * (sR[i] - gam * kh);
+            sQH[i] = gam * qh;
+        }
+        __syncthreads();
+        // ---- T = (I + A)^-1, one column per thread, column kept in registers
+        {
+            float tcol[C];
+            const int j = tid;
+            if (j < C) {
+#pragma unroll
+                for (int r = 0; r < C; ++r) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int s = 0; s < r; ++s) acc = fmaf(sA[r * CP + s], tcol[s], acc);
+                    tcol[r] = (r < j) ? 0.f : ((r == j) ? 1.f : -acc);
+                }
+            }
+            __syncthreads();
+            if (j < C) {
+#pragma unroll
+                for (int r = 0; r < C; ++r) sA[r * CP + j] = tcol[r];
+            }
+        }
+        __syncthreads();
+        // ---- Ut = T R
+        for (int i = tid; i < C * VS; i += nth) {
+            const int r = i / VS, j = i - r * VS;
+            float acc = 0.f;
+            for (int s = 0; s <= r; ++s) acc = fmaf(sA[r * CP + s], sR[s * VS + j], acc);
+            sU[i] = acc;
+        }
+        __syncthreads();
+        // ---- output rows of this chunk
+        for (int i = tid; i < C * VS; i += nth) {
+            const int r = i / VS, j = i - r * VS;
+            if (r < len) {
+                float acc = sQH[i];
+                for (int s = 0; s <= r; ++s) acc = fmaf(sP[r * CP + s], sU[s * VS + j], acc);
+                o[((t0 + r) * H + head) * (int64_t)V + v0 + j] = from_f32<TOut>(a.scale * acc);
+            }
+        }
+        // ---- state update
+        const float eL = expf(GL);
+        for (int i = tid; i < K * VS; i += nth) {
+            const int c = i / VS, j = i - c * VS;
+            float acc = 0.f;
+            for (int r = 0; r < C; ++r) acc = fmaf(sW[r] * sK[r * KP + c], sU[r * VS + j], acc);
+            sH[i] = fmaf(eL, sH[i], acc);
+        }
+    }
+    __syncthreads();
+    if (a.hT) {
+        for (int i = tid; i < K * VS; i += nth) {
+            const int c = i / VS, j = i - c * VS;
+            a.hT[hbase + (int64_t)c * V + v0 + j] = sH[i];
+        }
+    }
+}
+
+// ------------------------------------------------------------- schedule map
+// Packed batches: order the sequences longest first (ties by index) so that
+// the blocks of long sequences start first.  One block; rank by counting.
+// Writes order[n_seq] (int32) into the caller's workspace.
+__global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restrict__ cu, int n_seq,
+                                                        int32_t* __restrict__ order) {
+    for (int i = threadIdx.x; i < n_seq; i += blockDim.x) {
+        const int li = cu[i + 1] - cu[i];
+        int rank = 0;
+        for (int j = 0; j < n_seq; ++j) {
+            const int lj = cu[j + 1] - cu[j];
+            rank += (lj > li) || (lj == li && j < i);
+        }
+        order[rank] = i;
+    }
+}
+
+}  // namespace gdn

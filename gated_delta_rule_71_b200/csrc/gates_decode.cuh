@@ -1,0 +1,231 @@
+// gates_decode.cuh -- gate preparation and the Gated Delta Product decode step.
+//
+// Gates: Megatron-Core "core.ssm.ops.gdp.decode_prepare", module description and
+// the `softplus` entry.  Decode layout: the `gdp_decode_prepare` function entry
+// (post-conv row [value | key | query], ba row [b | a], outputs [n, M, H, *]).
+// The state update is the gated delta rule run over the M Householder copies.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdn {
+
+// ---------------------------------------------------------------- gate prep
+// Elementwise over [n_tok, H]; grid-stride.  HBM-bound (16 B in, 8 B out per
+// element), negligible next to the chunked pass.
+__global__ void __launch_bounds__(256) gate_prep_kernel(const float* __restrict__ a,
+                                                        const float* __restrict__ b,
+                                                        int64_t n_tok, int H, int64_t a_stride,
+                                                        int64_t b_stride,
+                                                        const float* __restrict__ A_log,
+                                                        const float* __restrict__ dt_bias,
+                                                        float* __restrict__ beta,
+                                                        float* __restrict__ g) {
+    const int64_t total = n_tok * H;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / H;
+        const int h = (int)(i - t * H);
+        g[i] = decay_gate(a[t * a_stride + h], dt_bias[h], A_log[h]);
+        beta[i] = write_gate(b[t * b_stride + h]);
+    }
+}
+
+// ------------------------------------------------------------- decode prepare
+// One block per (request, Householder copy).  Copies move in 16-byte units when
+// every source/destination offset is 16-byte aligned (VEC), else per element.
+template <bool VEC>
+__global__ void __launch_bounds__(256) gdp_prepare_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t xs, const __nv_bfloat16* __restrict__ ba,
+    int64_t bas, const float* __restrict__ A_log, const float* __restrict__ dt_bias, int M, int H,
+    int G, int P, int N, __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ k,
+    __nv_bfloat16* __restrict__ v, float* __restrict__ beta, float* __restrict__ g) {
+    const int r = blockIdx.x, m = blockIdx.y;
+    const int hpg = H / G;
+    const __nv_bfloat16* xr = x + (int64_t)r * xs;
+    const __nv_bfloat16* br = ba + (int64_t)r * bas;
+    const int64_t kbase = (int64_t)M * H * P, qbase = kbase + (int64_t)M * G * N;
+    const int64_t orow = (int64_t)r * M + m;  // [n, M] row of every output
+    using U = typename std::conditional<VEC, uint4, uint16_t>::type;
+    constexpr int E = sizeof(U) / 2;  // bf16 elements per unit
+    // value: the H*P slab of copy m is contiguous in x and in v
+    {
+        const U* src = reinterpret_cast<const U*>(xr + (int64_t)m * H * P);
+        U* dst = reinterpret_cast<U*>(v + orow * H * P);
+        for (int i = threadIdx.x; i < H * P / E; i += blockDim.x) dst[i] = src[i];
+    }
+    // key and query: head h reads group h / hpg
+    const int nN = N / E;
+    for (int i = threadIdx.x; i < H * nN; i += blockDim.x) {
+        const int h = i / nN, c = i - h * nN, grp = h / hpg;
+        const U* ks = reinterpret_cast<const U*>(xr + kbase + ((int64_t)m * G + grp) * N);
+        reinterpret_cast<U*>(k + (orow * H + h) * N)[c] = ks[c];
+        U qv;
+        if (m == M - 1) {
+            qv = reinterpret_cast<const U*>(xr + qbase + (int64_t)grp * N)[c];
+        } else {
+            memset(&qv, 0, sizeof(U));
+        }
+        reinterpret_cast<U*>(q + (orow * H + h) * N)[c] = qv;
+    }
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        beta[orow * H + h] = write_gate(__bfloat162float(br[m * H + h]));
+        g[orow * H + h] =
+            (m == 0) ? decay_gate(__bfloat162float(br[M * H + h]), dt_bias[h], A_log[h]) : 0.0f;
+    }
+}
+
+// ---------------------------------------------------------------- decode step
+// One block (8 warps) per (request, head).  The fp32 state [N, P] lives in
+// registers: warp w owns key rows [w*N/8, (w+1)*N/8), lane l owns value
+// columns [l*P/32, (l+1)*P/32), so every row is read and written as one
+// coalesced 512-byte (P = 128) warp access.  Column reductions over the key
+// axis go through shared memory.  The state is read once and written once:
+// the kernel is HBM-bound on 2*N*P*4 bytes per (request, head).
+constexpr int kDecWarps = 8;
+constexpr int kDecMaxM = 8;
+
+template <int N, int P>
+__global__ void __launch_bounds__(256) gdp_step_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t xs, const __nv_bfloat16* __restrict__ ba,
+    int64_t bas, const float* __restrict__ A_log, const float* __restrict__ dt_bias, int M, int H,
+    int G, float* __restrict__ state, __nv_bfloat16* __restrict__ o, float scale, int l2) {
+    constexpr int RPW = N / kDecWarps;  // rows per warp
+    constexpr int CPL = P / 32;         // columns per lane
+    __shared__ float kv[kDecMaxM][N];
+    __shared__ float vv[kDecMaxM][P];
+    __shared__ float qv[N];
+    __shared__ float red[kDecWarps][P];
+    __shared__ float uu[P];
+    __shared__ float gate_b[kDecMaxM];
+    __shared__ float gate_e;
+
+    const int rh = blockIdx.x;  // request * H + head
+    const int r = rh / H, h = rh - r * H;
+    const int hpg = H / G, grp = h / hpg;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const __nv_bfloat16* xr = x + (int64_t)r * xs;
+    const __nv_bfloat16* br = ba + (int64_t)r * bas;
+    const int64_t kbase = (int64_t)M * H * P, qbase = kbase + (int64_t)M * G * N;
+
+    // 1. issue the state loads first (the only large traffic)
+    float* st = state + (int64_t)rh * N * P;
+    float s[RPW][CPL];
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+        const float* src = st + (int64_t)(warp * RPW + rr) * P + lane * CPL;
+        if constexpr (CPL == 4) {
+            float4 t = *reinterpret_cast<const float4*>(src);
+            s[rr][0] = t.x; s[rr][1] = t.y; s[rr][2] = t.z; s[rr][3] = t.w;
+        } else if constexpr (CPL == 2) {
+            float2 t = *reinterpret_cast<const float2*>(src);
+            s[rr][0] = t.x; s[rr][1] = t.y;
+        } else {
+            s[rr][0] = src[0];
+        }
+    }
+
+    // 2. split / GQA-expand / normalise the M copies and the query into smem
+    for (int m = warp; m <= M; m += kDecWarps) {
+        const __nv_bfloat16* src = (m < M) ? xr + kbase + ((int64_t)m * G + grp) * N
+                                           : xr + qbase + (int64_t)grp * N;
+        float e[N / 32];
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < N / 32; ++i) {
+            e[i] = __bfloat162float(src[lane + 32 * i]);
+            ss = fmaf(e[i], e[i], ss);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv = l2 ? 1.0f / sqrtf(ss + 1e-6f) : 1.0f;
+        float* dst = (m < M) ? kv[m] : qv;
+#pragma unroll
+        for (int i = 0; i < N / 32; ++i) dst[lane + 32 * i] = e[i] * inv;
+    }
+    for (int i = threadIdx.x; i < M * P; i += blockDim.x) {
+        const int m = i / P, j = i - m * P;
+        vv[m][j] = __bfloat162float(xr[((int64_t)m * H + h) * P + j]);
+    }
+    if (threadIdx.x < M) gate_b[threadIdx.x] = write_gate(__bfloat162float(br[threadIdx.x * H + h]));
+    if (threadIdx.x == M)
+        gate_e = __double2float_rn(
+            exp((double)decay_gate(__bfloat162float(br[M * H + h]), dt_bias[h], A_log[h])));
+    __syncthreads();
+
+    // 3. the rule over the copies (decay on copy 0 only)
+    for (int m = 0; m < M; ++m) {
+        if (m == 0) {
+            const float e0 = gate_e;
+#pragma unroll
+            for (int rr = 0; rr < RPW; ++rr)
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) s[rr][c] *= e0;
+        }
+        float p[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) p[c] = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < RPW; ++rr) {
+            const float kk = kv[m][warp * RPW + rr];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) p[c] = fmaf(s[rr][c], kk, p[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = p[c];
+        __syncthreads();
+        if (threadIdx.x < P) {
+            float d = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) d += red[w][threadIdx.x];
+            uu[threadIdx.x] = gate_b[m] * (vv[m][threadIdx.x] - d);
+        }
+        __syncthreads();
+        float u[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) u[c] = uu[lane * CPL + c];
+#pragma unroll
+        for (int rr = 0; rr < RPW; ++rr) {
+            const float kk = kv[m][warp * RPW + rr];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) s[rr][c] = fmaf(kk, u[c], s[rr][c]);
+        }
+    }
+
+    // 4. output at the last copy: o = scale * S^T q
+    {
+        float p[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) p[c] = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < RPW; ++rr) {
+            const float qq = qv[warp * RPW + rr];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) p[c] = fmaf(s[rr][c], qq, p[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = p[c];
+        __syncthreads();
+        if (threadIdx.x < P) {
+            float d = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) d += red[w][threadIdx.x];
+            o[(int64_t)rh * P + threadIdx.x] = __float2bfloat16_rn(scale * d);
+        }
+    }
+
+    // 5. write the state back in place
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) {
+        float* dst = st + (int64_t)(warp * RPW + rr) * P + lane * CPL;
+        if constexpr (CPL == 4) {
+            *reinterpret_cast<float4*>(dst) = make_float4(s[rr][0], s[rr][1], s[rr][2], s[rr][3]);
+        } else if constexpr (CPL == 2) {
+            *reinterpret_cast<float2*>(dst) = make_float2(s[rr][0], s[rr][1]);
+        } else {
+            dst[0] = s[rr][0];
+        }
+    }
+}
+
+}  // namespace gdn

@@ -1,0 +1,270 @@
+// gdn_lib.cu -- the C ABI of libgdn.so (declared in include/gdn.h): host-side
+// argument checks, kernel selection and launches.  One translation unit holds
+// every kernel so that the device status word is a single symbol.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <type_traits>
+
+#include "gdn.h"
+#include "common.cuh"
+#include "gates_decode.cuh"
+#include "chunk_simt.cuh"
+#include "chunk_tc.cuh"
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+gdn_status cuda_check(cudaError_t e) {
+    if (e == cudaSuccess) return GDN_OK;
+    t_last_cuda_error = (int)e;
+    return GDN_ERR_CUDA;
+}
+
+gdn_status launch_check() { return cuda_check(cudaGetLastError()); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+// ------------------------------------------------------------- chunk (fp32)
+
+template <int C, typename TIn, typename TOut>
+gdn_status launch_simt(const gdn::ChunkArgs& a, int n_blocks, cudaStream_t st) {
+    const size_t smem = (size_t)gdn::simt_smem_floats(C, a.K, a.VS) * sizeof(float);
+    auto kern = gdn::chunk_fwd_simt_kernel<C, TIn, TOut>;
+    gdn_status s = cuda_check(
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    if (s != GDN_OK) return s;
+    kern<<<n_blocks, 256, smem, st>>>(a);
+    return launch_check();
+}
+
+template <int C>
+gdn_status launch_simt_dt(const gdn::ChunkArgs& a, gdn_dtype in, gdn_dtype out, int nb,
+                          cudaStream_t st) {
+    using bf = __nv_bfloat16;
+    if (in == GDN_F32 && out == GDN_F32) return launch_simt<C, float, float>(a, nb, st);
+    if (in == GDN_F32 && out == GDN_BF16) return launch_simt<C, float, bf>(a, nb, st);
+    if (in == GDN_BF16 && out == GDN_F32) return launch_simt<C, bf, float>(a, nb, st);
+    return launch_simt<C, bf, bf>(a, nb, st);
+}
+
+constexpr size_t kSimtSmemMax = 227 * 1024;
+
+size_t ws_schedule_bytes(int n_seq) { return ((size_t)n_seq * 4 + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(int s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: argument rejected on the host";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: size or dtype not built";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA call or launch failed";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a bounded device wait gave up";
+        default: return "unknown gdn_status";
+    }
+}
+
+int gdn_last_cuda_error(void) { return t_last_cuda_error; }
+
+int gdn_version(void) { return 100; }
+
+gdn_status gdn_gate_prep(const float* a, const float* b, int64_t n_tok, int H, int64_t a_stride,
+                         int64_t b_stride, const float* A_log, const float* dt_bias, float* beta,
+                         float* g, void* stream) {
+    if (n_tok < 0 || H < 1 || a_stride < H || b_stride < H) return GDN_ERR_INVALID_ARG;
+    if (n_tok == 0) return GDN_OK;
+    if (!a || !b || !A_log || !dt_bias || !beta || !g) return GDN_ERR_INVALID_ARG;
+    const int64_t total = n_tok * H;
+    const int64_t want = (total + 255) / 256;
+    const int blocks = (int)(want < (int64_t)num_sms() * 16 ? want : (int64_t)num_sms() * 16);
+    gdn::gate_prep_kernel<<<blocks, 256, 0, as_stream(stream)>>>(a, b, n_tok, H, a_stride,
+                                                                 b_stride, A_log, dt_bias, beta, g);
+    return launch_check();
+}
+
+size_t gdn_chunk_fwd_workspace_size(int n_seq, int64_t T_total, int H, int K, int V,
+                                    gdn_dtype qkv_dtype) {
+    (void)T_total; (void)H; (void)K; (void)V; (void)qkv_dtype;
+    // the packed-batch schedule (one int32 per sequence)
+    return n_seq > 0 ? ws_schedule_bytes(n_seq) : 0;
+}
+
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype qkv_dtype,
+                         const float* g, const float* beta, const float* h0,
+                         const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int H, int K,
+                         int V, float scale, void* o, gdn_dtype o_dtype, float* hT,
+                         void* workspace, size_t ws_bytes, unsigned flags, void* stream) {
+    if (B < 0 || T < 0 || H < 1 || n_seq < 0) return GDN_ERR_INVALID_ARG;
+    if ((qkv_dtype != GDN_F32 && qkv_dtype != GDN_BF16) ||
+        (o_dtype != GDN_F32 && o_dtype != GDN_BF16))
+        return GDN_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (B != 1) return GDN_ERR_INVALID_ARG;
+    } else {
+        n_seq = B;
+    }
+    if (!head_dim_ok(K) || !head_dim_ok(V)) return GDN_ERR_UNSUPPORTED;
+    if (n_seq == 0) return GDN_OK;
+    if (B * T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
+    for (const void* p : {q, k, v, (const void*)g, (const void*)beta, (const void*)h0,
+                          (const void*)o, (const void*)hT, (const void*)cu_seqlens})
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t ws_need = cu_seqlens ? ws_schedule_bytes(n_seq) : 0;
+    if (ws_need && (!workspace || ws_bytes < ws_need || !aligned16(workspace)))
+        return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && (int64_t)n_seq * T * H > ((int64_t)1 << 40)) return GDN_ERR_UNSUPPORTED;
+
+    cudaStream_t st = as_stream(stream);
+    const int32_t* order = nullptr;
+    if (cu_seqlens && n_seq > 1) {
+        int32_t* ord = static_cast<int32_t*>(workspace);
+        gdn::schedule_kernel<<<1, 1024, 0, st>>>(cu_seqlens, n_seq, ord);
+        gdn_status s = launch_check();
+        if (s != GDN_OK) return s;
+        order = ord;
+    }
+
+    gdn::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0;
+    a.cu_seqlens = cu_seqlens; a.order = order; a.n_seq = n_seq; a.T = T;
+    a.H = H; a.K = K; a.V = V; a.scale = scale; a.o = o; a.hT = hT;
+
+    int nvs_forced = (flags & GDN_FLAG_VSPLIT1) ? 1 : (flags & GDN_FLAG_VSPLIT2) ? 2
+                   : (flags & GDN_FLAG_VSPLIT4) ? 4 : 0;
+
+    const bool tc_ok = gdn::kTcAvailable && qkv_dtype == GDN_BF16 && K == 128 && V == 128 &&
+                       !(flags & (GDN_FLAG_EXACT_F32 | GDN_FLAG_CHUNK16 | GDN_FLAG_CHUNK32));
+    if (tc_ok) {
+        int nvs = nvs_forced ? nvs_forced : 2;
+        if (nvs != 1 && nvs != 2) return GDN_ERR_UNSUPPORTED;
+        a.nvs = nvs;
+        a.VS = V / nvs;
+        return gdn::launch_chunk_tc(a, o_dtype == GDN_BF16, st) == 0 ? launch_check()
+                                                                     : GDN_ERR_UNSUPPORTED;
+    }
+
+    const int C = (flags & GDN_FLAG_CHUNK16) ? 16 : (flags & GDN_FLAG_CHUNK32) ? 32 : 64;
+    int nvs = nvs_forced ? nvs_forced : (V > 32 ? V / 32 : 1);
+    if (V % nvs) return GDN_ERR_UNSUPPORTED;
+    a.nvs = nvs;
+    a.VS = V / nvs;
+    if ((size_t)gdn::simt_smem_floats(C, K, a.VS) * 4 > kSimtSmemMax) return GDN_ERR_UNSUPPORTED;
+    const int64_t nb = (int64_t)n_seq * H * nvs;
+    if (nb > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    if (C == 16) return launch_simt_dt<16>(a, qkv_dtype, o_dtype, (int)nb, st);
+    if (C == 32) return launch_simt_dt<32>(a, qkv_dtype, o_dtype, (int)nb, st);
+    return launch_simt_dt<64>(a, qkv_dtype, o_dtype, (int)nb, st);
+}
+
+static gdn_status decode_args_ok(const void* x, int64_t xs, const void* ba, int64_t bas,
+                                 const float* A_log, const float* dt_bias, int n, int M, int H,
+                                 int G, int P, int N) {
+    if (n < 0 || M < 1 || H < 1 || G < 1 || H % G) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(P) || !head_dim_ok(N)) return GDN_ERR_UNSUPPORTED;
+    const int64_t row = (int64_t)M * H * P + (int64_t)M * G * N + (int64_t)G * N;
+    if (xs < row || bas < (int64_t)M * H + H) return GDN_ERR_INVALID_ARG;
+    if (n > 0 && (!x || !ba || !A_log || !dt_bias)) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+gdn_status gdp_decode_prepare(const void* x, int64_t x_n_stride, const void* ba,
+                              int64_t ba_n_stride, const float* A_log, const float* dt_bias, int n,
+                              int M, int H, int G, int P, int N, void* q, void* k, void* v,
+                              float* beta, float* g, void* stream) {
+    gdn_status s = decode_args_ok(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P, N);
+    if (s != GDN_OK) return s;
+    if (n == 0) return GDN_OK;
+    if (!q || !k || !v || !beta || !g) return GDN_ERR_INVALID_ARG;
+    if (M > 65535) return GDN_ERR_UNSUPPORTED;
+    const bool vec = aligned16(x) && aligned16(q) && aligned16(k) && aligned16(v) &&
+                     (x_n_stride % 8) == 0;
+    using bf = __nv_bfloat16;
+    dim3 grid(n, M);
+    if (vec)
+        gdn::gdp_prepare_kernel<true><<<grid, 256, 0, as_stream(stream)>>>(
+            (const bf*)x, x_n_stride, (const bf*)ba, ba_n_stride, A_log, dt_bias, M, H, G, P, N,
+            (bf*)q, (bf*)k, (bf*)v, beta, g);
+    else
+        gdn::gdp_prepare_kernel<false><<<grid, 256, 0, as_stream(stream)>>>(
+            (const bf*)x, x_n_stride, (const bf*)ba, ba_n_stride, A_log, dt_bias, M, H, G, P, N,
+            (bf*)q, (bf*)k, (bf*)v, beta, g);
+    return launch_check();
+}
+
+gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, int64_t ba_n_stride,
+                           const float* A_log, const float* dt_bias, int n, int M, int H, int G,
+                           int P, int N, float* state, void* o, float scale, int qk_l2norm,
+                           void* stream) {
+    gdn_status s = decode_args_ok(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P, N);
+    if (s != GDN_OK) return s;
+    if (n == 0) return GDN_OK;
+    if (!state || !o || !aligned16(state)) return GDN_ERR_INVALID_ARG;
+    if (M > gdn::kDecMaxM) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)n * H > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    using bf = __nv_bfloat16;
+    const int nb = n * H;
+    cudaStream_t st = as_stream(stream);
+#define GDN_DEC(NN, PP)                                                                          \
+    if (N == NN && P == PP) {                                                                    \
+        gdn::gdp_step_kernel<NN, PP><<<nb, 256, 0, st>>>((const bf*)x, x_n_stride, (const bf*)ba, \
+                                                          ba_n_stride, A_log, dt_bias, M, H, G,  \
+                                                          state, (bf*)o, scale, qk_l2norm);      \
+        return launch_check();                                                                   \
+    }
+    GDN_DEC(128, 128) GDN_DEC(128, 64) GDN_DEC(128, 32)
+    GDN_DEC(64, 128) GDN_DEC(64, 64) GDN_DEC(64, 32)
+    GDN_DEC(32, 128) GDN_DEC(32, 64) GDN_DEC(32, 32)
+#undef GDN_DEC
+    return GDN_ERR_UNSUPPORTED;
+}
+
+gdn_status gdn_device_status(void* stream) {
+    cudaStream_t st = as_stream(stream);
+    unsigned int word = 0, zero = 0;
+    gdn_status s = cuda_check(cudaMemcpyFromSymbolAsync(&word, gdn::g_status_word, sizeof(word), 0,
+                                                        cudaMemcpyDeviceToHost, st));
+    if (s != GDN_OK) return s;
+    s = cuda_check(cudaMemcpyToSymbolAsync(gdn::g_status_word, &zero, sizeof(zero), 0,
+                                           cudaMemcpyHostToDevice, st));
+    if (s != GDN_OK) return s;
+    s = cuda_check(cudaStreamSynchronize(st));
+    if (s != GDN_OK) return s;
+    return (gdn_status)word;
+}
+
+}  // extern "C"
+
+namespace gdn {
+__global__ void selftest_wait_kernel(unsigned polls) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, polls);  // nothing ever arrives
+    __syncthreads();
+}
+}  // namespace gdn
+
+extern "C" gdn_status gdn_selftest_wait_timeout(unsigned polls, void* stream) {
+    if (polls == 0 || polls > (1u << 20)) return GDN_ERR_INVALID_ARG;
+    gdn::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(polls);
+    return launch_check();
+}

@@ -1,0 +1,196 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the gated delta rule (chunked forward) and the
+ * Gated Delta Product one-token decode step on NVIDIA B200 (sm_100a).
+ *
+ * The rule (per sequence, per head; S is V x K, the library stores h = S^T,
+ * K x V, key-major):
+ *     S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = scale * S_t q_t
+ * Chunked evaluation (64-token chunks, intra-chunk WY form, inter-chunk state
+ * recurrence, chunk output) follows the three GDN kernels of ZzCompute,
+ * PyTorch Helion Hackathon gallery entry 11, items 2-4 ("Chunk Forward H",
+ * "Chunk Forward O", "Recompute W/U").  Gates and the decode layout follow
+ * NVIDIA Megatron-Core "core.ssm.ops.gdp.decode_prepare".
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers to memory the caller owns.  The
+ *    library never allocates, never frees, never synchronises the host with
+ *    the device (except gdn_device_status, which says so) and keeps no state
+ *    between calls apart from the device status word.
+ *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  Work is enqueued on it and the call returns; results are ready
+ *    when the stream reaches that point.  No call reads device memory on the
+ *    host, so every call may be captured in a CUDA graph.
+ *  - Arguments are checked on the host before anything is launched; a bad
+ *    argument returns GDN_ERR_INVALID_ARG and launches nothing.  A failed
+ *    launch returns GDN_ERR_CUDA (gdn_last_cuda_error gives the cudaError_t).
+ *  - Layouts are row-major with the innermost dimension contiguous unless a
+ *    stride argument says otherwise.  Every output element is written by
+ *    exactly one thread, with no atomics, so results are bitwise reproducible
+ *    run to run on the same device.
+ *  - Pointers must be 16-byte aligned (256-byte alignment, as from the CUDA
+ *    caching allocators, is recommended).
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1, /* rejected on the host; nothing launched            */
+    GDN_ERR_UNSUPPORTED = 2, /* well-formed, but this size/dtype is not built     */
+    GDN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed              */
+    GDN_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (device status) */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* gdn_chunk_fwd flags (bit set). */
+#define GDN_FLAG_EXACT_F32 0x1u    /* use the fp32-FMA kernel even for bf16 q/k/v      */
+#define GDN_FLAG_CHUNK32 0x10u     /* fp32-FMA kernel only: 32-token chunks           */
+#define GDN_FLAG_CHUNK16 0x20u     /* fp32-FMA kernel only: 16-token chunks           */
+#define GDN_FLAG_VSPLIT1 0x100u    /* force one V-slice per (sequence, head)          */
+#define GDN_FLAG_VSPLIT2 0x200u    /* force two V-slices                              */
+#define GDN_FLAG_VSPLIT4 0x400u    /* force four V-slices                             */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gdn_status_string(int status);
+
+/* cudaError_t of the most recent GDN_ERR_CUDA on the calling thread (0 if none). */
+int gdn_last_cuda_error(void);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int gdn_version(void);
+
+/*
+ * gdn_gate_prep -- per-token, per-head gates.
+ *   beta = sigmoid(b)
+ *   g    = -exp(A_log) * softplus(a + dt_bias),
+ *   softplus(x) = log1p(exp(x)), and x itself when x > 20 (strict).
+ * Megatron-Core "core.ssm.ops.gdp.decode_prepare", module description and the
+ * `softplus` entry (torch's F.softplus at beta = 1, threshold 20; log1p keeps
+ * the far-negative tail).  a + dt_bias is one fp32 add; the transcendentals
+ * run in fp64 and each output is rounded to fp32 once (no flush to zero).
+ *
+ *   a, b      : fp32 [n_tok, H], token stride a_stride / b_stride elements
+ *               (>= H), head stride 1.
+ *   A_log     : fp32 [H].   dt_bias : fp32 [H].
+ *   beta, g   : fp32 [n_tok, H] contiguous, written.
+ * n_tok == 0 is a no-op.  Errors: INVALID_ARG for NULL pointers, H < 1,
+ * n_tok < 0 or a stride < H.
+ */
+gdn_status gdn_gate_prep(const float* a, const float* b, int64_t n_tok, int H, int64_t a_stride,
+                         int64_t b_stride, const float* A_log, const float* dt_bias, float* beta,
+                         float* g, void* stream);
+
+/*
+ * gdn_chunk_fwd_workspace_size -- bytes of device workspace gdn_chunk_fwd
+ * needs for these sizes (0 for a dense batch).  The caller allocates it.
+ */
+size_t gdn_chunk_fwd_workspace_size(int n_seq, int64_t T_total, int H, int K, int V,
+                                    gdn_dtype qkv_dtype);
+
+/*
+ * gdn_chunk_fwd -- chunked forward pass of the gated delta rule.
+ *
+ *   q, k    : [B, T, H, K] of qkv_dtype (GDN_F32 or GDN_BF16).
+ *   v       : [B, T, H, V] of qkv_dtype.
+ *   g, beta : fp32 [B, T, H] (natural-log decay gate, write strength).
+ *   h0      : fp32 [n_seq, H, K, V] initial states, or NULL for zeros.
+ *   cu_seqlens : NULL for a dense batch (n_seq = B sequences of length T), or
+ *             int32 [n_seq + 1] device array of packed-sequence offsets with
+ *             cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seq] = T; then
+ *             B must be 1.  Empty sequences are allowed (their h_T = h0).
+ *   scale   : multiplies every output (o_t = scale * S_t q_t).
+ *   o       : [B, T, H, V] of o_dtype (GDN_F32 or GDN_BF16), written.
+ *   hT      : fp32 [n_seq, H, K, V] final states, written; NULL to skip.
+ *   workspace / ws_bytes : device scratch of at least
+ *             gdn_chunk_fwd_workspace_size(...) bytes (may be NULL when that
+ *             is 0).  Its contents on entry do not matter.
+ *   flags   : GDN_FLAG_* bits; 0 selects the fastest kernel for the dtype.
+ * Supported: K, V in {32, 64, 128}.  bf16 q/k/v run on the tcgen05 tensor-core
+ * kernel (bf16 operands, fp32 accumulation and fp32 state) when K = V = 128;
+ * otherwise, and for fp32 q/k/v, an fp32-FMA kernel that keeps every product
+ * in IEEE fp32.  T == 0 writes only hT (= h0 or zeros).
+ * Errors: INVALID_ARG (NULL q/k/v/g/beta/o, sizes < 0, B != 1 with
+ * cu_seqlens, workspace too small, misaligned pointer), UNSUPPORTED (other
+ * K/V/dtypes).  cu_seqlens contents are not checked on the host (that would
+ * need a device read); offsets outside [0, T] are undefined behaviour.
+ */
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype qkv_dtype,
+                         const float* g, const float* beta, const float* h0,
+                         const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int H, int K,
+                         int V, float scale, void* o, gdn_dtype o_dtype, float* hT,
+                         void* workspace, size_t ws_bytes, unsigned flags, void* stream);
+
+/*
+ * gdp_decode_prepare -- split, GQA-expand, Householder-interleave and gate one
+ * decode step.  Megatron-Core `gdp_decode_prepare` (function entry, parameter
+ * list and return shapes).
+ *
+ *   x   : bf16 [n, *] rows, row stride x_n_stride elements, each row
+ *         [value: M*H*P | key: M*G*N | query: G*N] (inner dim contiguous).
+ *   ba  : bf16 [n, *] rows, row stride ba_n_stride elements, each row
+ *         [b: M*H | a: H].
+ *   A_log, dt_bias : fp32 [H].
+ *   q, k : bf16 [n, M, H, N] written;  v : bf16 [n, M, H, P] written.
+ *   beta, g : fp32 [n, M, H] written.
+ * Readings where the page is silent: the Householder copy is the outer index
+ * inside each part ([M,H,P], [M,G,N], [M,H]); head h uses group h / (H/G);
+ * the query sits on copy M-1 (zeros elsewhere); the decay g sits on copy 0
+ * (zero elsewhere); beta is per copy.  q/k/v are bit copies of x; beta and g
+ * are computed as in gdn_gate_prep from the bf16 inputs widened to fp32.
+ * Errors: INVALID_ARG (NULL, n < 0, M < 1, H % G != 0, strides shorter than
+ * the row), UNSUPPORTED (P or N not in {32, 64, 128}).
+ */
+gdn_status gdp_decode_prepare(const void* x, int64_t x_n_stride, const void* ba,
+                              int64_t ba_n_stride, const float* A_log, const float* dt_bias, int n,
+                              int M, int H, int G, int P, int N, void* q, void* k, void* v,
+                              float* beta, float* g, void* stream);
+
+/*
+ * gdp_decode_step -- the fused decode step: gdp_decode_prepare's split, GQA
+ * expansion and gates in registers, then the rule over the M copies of each
+ * request, starting from and overwriting its state:
+ *     for m in 0..M-1:  S <- exp(g_m) S;  u = beta_m (v_m - S^T k_m);
+ *                       S <- S + k_m u^T
+ *     o = scale * S^T q_{M-1}
+ * (state layout [n, H, N, P]: key rows, value columns).  With qk_l2norm != 0
+ * every q and k vector is divided by sqrt(sum x^2 + 1e-6) first.
+ *   state : fp32 [n, H, N, P], read and written in place.
+ *   o     : bf16 [n, H, P], written.
+ * Other arguments and errors as gdp_decode_prepare.
+ */
+gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, int64_t ba_n_stride,
+                           const float* A_log, const float* dt_bias, int n, int M, int H, int G,
+                           int P, int N, float* state, void* o, float scale, int qk_l2norm,
+                           void* stream);
+
+/*
+ * gdn_device_status -- reads and clears the device status word on the current
+ * device.  Kernels that wait on the device (mbarrier waits in the tensor-core
+ * kernel) give up after a bounded number of polls, record GDN_ERR_TIMEOUT
+ * there and return, so the context stays usable.  This call SYNCHRONISES the
+ * stream.  Returns GDN_OK when nothing was recorded.
+ */
+gdn_status gdn_device_status(void* stream);
+
+/*
+ * gdn_selftest_wait_timeout -- launches one block that waits on an mbarrier
+ * nothing will ever complete, polling at most `polls` times, then records
+ * GDN_ERR_TIMEOUT in the device status word and returns.  Exercises the
+ * failure path of the bounded waits without hanging or faulting the device.
+ */
+gdn_status gdn_selftest_wait_timeout(unsigned polls, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

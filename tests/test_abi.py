@@ -1,0 +1,109 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry
+point, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_71_b200 import _lib
+from gated_delta_rule_71_b200.build import LIB, ROOT
+
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:gdn|gdp)_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exists_and_loads():
+    assert os.path.exists(LIB), "build the library first (__graft_entry__.build())"
+    _lib.load()
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(LIB)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in gdn.h but not exported"
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings():
+    lib = _lib.load()
+    for s in range(5):
+        assert lib.gdn_status_string(s).startswith(b"GDN_")
+    assert lib.gdn_status_string(99) == b"unknown gdn_status"
+    assert lib.gdn_version() >= 100
+
+
+INVALID = 1
+UNSUPPORTED = 2
+
+
+def test_gate_prep_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(16)  # never dereferenced: rejected first
+    assert lib.gdn_gate_prep(p, p, 10, 0, 4, 4, p, p, p, p, None) == INVALID
+    assert lib.gdn_gate_prep(p, p, -1, 4, 4, 4, p, p, p, p, None) == INVALID
+    assert lib.gdn_gate_prep(p, p, 10, 4, 3, 4, p, p, p, p, None) == INVALID
+    assert lib.gdn_gate_prep(None, p, 10, 4, 4, 4, p, p, p, p, None) == INVALID
+    assert lib.gdn_gate_prep(None, None, 0, 4, 4, 4, None, None, None, None, None) == 0
+
+
+def test_chunk_fwd_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    args = lambda **kw: [kw.get("q", p), p, p, kw.get("dt", 1), p, p, None, kw.get("cu", None),
+                         kw.get("n_seq", 0), kw.get("B", 2), kw.get("T", 64), kw.get("H", 2),
+                         kw.get("K", 128), kw.get("V", 128), 1.0, p, kw.get("odt", 0), p,
+                         kw.get("ws", None), kw.get("wsb", 0), 0, None]
+    assert lib.gdn_chunk_fwd(*args(K=96)) == UNSUPPORTED
+    assert lib.gdn_chunk_fwd(*args(V=256)) == UNSUPPORTED
+    assert lib.gdn_chunk_fwd(*args(dt=7)) == INVALID
+    assert lib.gdn_chunk_fwd(*args(odt=5)) == INVALID
+    assert lib.gdn_chunk_fwd(*args(q=None)) == INVALID
+    assert lib.gdn_chunk_fwd(*args(q=ctypes.c_void_p(258))) == INVALID  # misaligned
+    assert lib.gdn_chunk_fwd(*args(T=-1)) == INVALID
+    assert lib.gdn_chunk_fwd(*args(H=0)) == INVALID
+    # packed sequences need B == 1 and a workspace
+    assert lib.gdn_chunk_fwd(*args(cu=p, n_seq=3, B=2)) == INVALID
+    assert lib.gdn_chunk_fwd(*args(cu=p, n_seq=3, B=1)) == INVALID
+    assert lib.gdn_chunk_fwd_workspace_size(3, 100, 2, 128, 128, 1) >= 12
+    assert lib.gdn_chunk_fwd_workspace_size(0, 100, 2, 128, 128, 1) == 0
+    # no sequences: nothing to do
+    assert lib.gdn_chunk_fwd(*args(B=0)) == 0
+
+
+def test_decode_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    n, M, H, G, P, N = 4, 2, 32, 16, 128, 128
+    row = M * H * P + M * G * N + G * N
+    ok = [p, row, p, M * H + H, p, p, n, M, H, G, P, N]
+    assert lib.gdp_decode_prepare(*ok[:8], 31, *ok[9:], p, p, p, p, p, None) == INVALID  # H % G
+    assert lib.gdp_decode_prepare(p, row - 1, *ok[2:], p, p, p, p, p, None) == INVALID
+    assert lib.gdp_decode_prepare(p, row, p, M * H, *ok[4:], p, p, p, p, p, None) == INVALID
+    assert lib.gdp_decode_prepare(*ok[:10], 96, N, p, p, p, p, p, None) == UNSUPPORTED
+    assert lib.gdp_decode_step(*ok, None, p, 1.0, 1, None) == INVALID
+    assert lib.gdp_decode_step(p, row, p, M * H + H, p, p, n, 0, H, G, P, N, p, p, 1.0, 1,
+                               None) == INVALID
+    big = [p, 9 * H * P + 9 * G * N + G * N, p, 9 * H + H, p, p, n, 9, H, G, P, N]
+    assert lib.gdp_decode_step(*big, p, p, 1.0, 1, None) == UNSUPPORTED  # M > 8
+    assert lib.gdp_decode_step(*ok[:6], 0, *ok[7:], p, p, 1.0, 1, None) == 0  # n == 0
+
+
+def test_selftest_rejects_zero_polls():
+    assert _lib.load().gdn_selftest_wait_timeout(0, None) == INVALID
+
+
+def test_package_has_no_cpu_fallback():
+    # the binding never imports the oracle and has no torch compute path
+    pkg = os.path.join(ROOT, "gated_delta_rule_71_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert "import oracle" not in src and "from oracle" not in src, fn
