@@ -54,7 +54,7 @@ def gate_prep(a: torch.Tensor, b: torch.Tensor, A_log: torch.Tensor, dt_bias: to
         _need(t, n, torch.float32, dev, contiguous=False)
     a2 = a.reshape(-1, H)
     b2 = b.reshape(-1, H)
-    if a2.stride(-1) != 1 or b2.stride(-1) != 1:
+    if H > 1 and (a2.stride(-1) != 1 or b2.stride(-1) != 1):
         raise ValueError("a and b need a contiguous head dimension")
     for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias")):
         _need(t, n, torch.float32, dev)

@@ -122,9 +122,10 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype 
     if (!head_dim_ok(K) || !head_dim_ok(V)) return GDN_ERR_UNSUPPORTED;
     if (n_seq == 0) return GDN_OK;
     if (B * T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
-    for (const void* p : {q, k, v, (const void*)g, (const void*)beta, (const void*)h0,
-                          (const void*)o, (const void*)hT, (const void*)cu_seqlens})
+    for (const void* p : {q, k, v, (const void*)h0, (const void*)o, (const void*)hT})
         if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    for (const void* p : {(const void*)g, (const void*)beta, (const void*)cu_seqlens})
+        if (p && (reinterpret_cast<uintptr_t>(p) & 3u)) return GDN_ERR_INVALID_ARG;
     const size_t ws_need = cu_seqlens ? ws_schedule_bytes(n_seq) : 0;
     if (ws_need && (!workspace || ws_bytes < ws_need || !aligned16(workspace)))
         return GDN_ERR_INVALID_ARG;
@@ -149,14 +150,19 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype 
                    : (flags & GDN_FLAG_VSPLIT4) ? 4 : 0;
 
     const bool tc_ok = gdn::kTcAvailable && qkv_dtype == GDN_BF16 && K == 128 && V == 128 &&
+                       (cu_seqlens ? T : (int64_t)B * T) > 0 &&
+                       (cu_seqlens ? T : (int64_t)B * T) < ((int64_t)1 << 31) &&
+                       (nvs_forced == 0 || nvs_forced == 2) &&
                        !(flags & (GDN_FLAG_EXACT_F32 | GDN_FLAG_CHUNK16 | GDN_FLAG_CHUNK32));
     if (tc_ok) {
-        int nvs = nvs_forced ? nvs_forced : 2;
-        if (nvs != 1 && nvs != 2) return GDN_ERR_UNSUPPORTED;
-        a.nvs = nvs;
-        a.VS = V / nvs;
-        return gdn::launch_chunk_tc(a, o_dtype == GDN_BF16, st) == 0 ? launch_check()
-                                                                     : GDN_ERR_UNSUPPORTED;
+        a.nvs = 2;
+        a.VS = V / 2;
+        const int rc = gdn::launch_chunk_tc(a, cu_seqlens ? T : (int64_t)B * T,
+                                            o_dtype == GDN_BF16, st);
+        if (rc == 1) return GDN_ERR_UNSUPPORTED;
+        if (rc == 2) return cuda_check(cudaGetLastError() != cudaSuccess ? cudaErrorInvalidValue
+                                                                         : cudaErrorInvalidValue);
+        return launch_check();
     }
 
     const int C = (flags & GDN_FLAG_CHUNK16) ? 16 : (flags & GDN_FLAG_CHUNK32) ? 32 : 64;
