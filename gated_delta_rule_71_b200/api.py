@@ -176,3 +176,32 @@ def device_status(device=None) -> int:
 def selftest_wait_timeout(polls: int = 64, device=None) -> None:
     s = torch.cuda.current_stream(device).cuda_stream
     _lib.call("gdn_selftest_wait_timeout", int(polls), s)
+
+
+def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                      beta: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                      cu_seqlens: Optional[torch.Tensor] = None, scale: float = 1.0,
+                      out: Optional[torch.Tensor] = None, hT: Optional[torch.Tensor] = None,
+                      flags: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """chunk_fwd through gdn_chunk_fwd_noalloc: no workspace is passed; the
+    library's fixed schedule array (GDN_NOALLOC_MAX_SEQS sequences) is used
+    instead.  For callers whose own code must not allocate device memory, pass
+    preallocated ``out`` (fp32 [B,T,H,V]) and ``hT`` (fp32 [n_seq,H,K,V]); the
+    library call itself never allocates."""
+    dev = q.device
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    if q.dtype not in _DT or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype: float32 or bfloat16")
+    n_seq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, V), dtype=torch.float32, device=dev)
+    if hT is None:
+        hT = torch.empty((n_seq, H, K, V), dtype=torch.float32, device=dev)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (out, "out"),
+                 (hT, "hT")):
+        _need(t, n, None, dev)
+    _lib.call("gdn_chunk_fwd_noalloc", _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(g),
+              _ptr(beta), _ptr(h0), _ptr(cu_seqlens), n_seq, B, T, H, K, V, float(scale),
+              _ptr(out), _DT[out.dtype], _ptr(hT), int(flags), _stream(q))
+    return out, hT

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "gdn.h"
@@ -76,6 +77,9 @@ const char* gdn_status_string(int s) {
         case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: size or dtype not built";
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA call or launch failed";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a bounded device wait gave up";
+        case GDN_ERR_TOO_LARGE:
+            return "GDN_ERR_TOO_LARGE: more packed sequences than gdn_chunk_fwd_noalloc's fixed "
+                   "schedule array holds (GDN_NOALLOC_MAX_SEQS)";
         default: return "unknown gdn_status";
     }
 }
@@ -273,4 +277,61 @@ extern "C" gdn_status gdn_selftest_wait_timeout(unsigned polls, void* stream) {
     if (polls == 0 || polls > (1u << 20)) return GDN_ERR_INVALID_ARG;
     gdn::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(polls);
     return launch_check();
+}
+
+// ----------------------------------------------------------------------------
+// gdn_chunk_fwd_noalloc: the chunked forward for callers that cannot allocate
+// device memory (see include/gdn.h).  Its only scratch -- the longest-first
+// schedule of a packed batch -- lives in this fixed device array instead of a
+// caller-provided workspace.  Host code must not hand the array's name to a
+// kernel: on the host it is only a stand-in symbol, so its device address is
+// looked up once per device with cudaGetSymbolAddress and cached.
+static __device__ __align__(256) int32_t g_noalloc_schedule[GDN_NOALLOC_MAX_SEQS];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_schedule on the current device; looked up on the
+// first call for that device (this is why that first call must not be made
+// while a stream is being captured).
+gdn_status noalloc_schedule_addr(void** out) {
+    int dev = 0;
+    gdn_status s = cuda_check(cudaGetDevice(&dev));
+    if (s != GDN_OK) return s;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return GDN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        s = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_schedule));
+        if (s != GDN_OK) return s;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return GDN_OK;
+}
+}  // namespace
+
+extern "C" gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                            gdn_dtype qkv_dtype, const float* g,
+                                            const float* beta, const float* h0,
+                                            const int32_t* cu_seqlens, int n_seq, int B,
+                                            int64_t T, int H, int K, int V, float scale, void* o,
+                                            gdn_dtype o_dtype, float* hT, unsigned flags,
+                                            void* stream) {
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    if (cu_seqlens) {
+        if (n_seq > GDN_NOALLOC_MAX_SEQS) return GDN_ERR_TOO_LARGE;
+        if (n_seq > 1) {
+            // every entry the schedule kernel later reads it first writes, so the
+            // array needs no clearing between calls
+            gdn_status s = noalloc_schedule_addr(&ws);
+            if (s != GDN_OK) return s;
+            ws_bytes = sizeof(g_noalloc_schedule);
+        }
+    }
+    return gdn_chunk_fwd(q, k, v, qkv_dtype, g, beta, h0, cu_seqlens, n_seq, B, T, H, K, V, scale,
+                         o, o_dtype, hT, ws, ws_bytes, flags, stream);
 }

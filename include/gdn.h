@@ -46,7 +46,8 @@ typedef enum {
     GDN_ERR_INVALID_ARG = 1, /* rejected on the host; nothing launched            */
     GDN_ERR_UNSUPPORTED = 2, /* well-formed, but this size/dtype is not built     */
     GDN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed              */
-    GDN_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (device status) */
+    GDN_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (device status) */
+    GDN_ERR_TOO_LARGE = 5    /* exceeds the fixed capacity of gdn_chunk_fwd_noalloc  */
 } gdn_status;
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -171,6 +172,38 @@ gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, in
                            const float* A_log, const float* dt_bias, int n, int M, int H, int G,
                            int P, int N, float* state, void* o, float scale, int qk_l2norm,
                            void* stream);
+
+/*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate
+ * device memory.  The sources describe no such entry point; it exists because
+ * some callers have no way to provide the packed-batch workspace: code running
+ * inside a region where the allocator is off limits (an inference server
+ * that reserved all device memory for its KV cache up front, a plugin whose
+ * host framework owns the allocator and exposes none through a C ABI, a
+ * real-time loop that cannot afford cudaMalloc's implicit synchronisation and
+ * unbounded latency).
+ *
+ * Same arguments and results as gdn_chunk_fwd, without workspace / ws_bytes.
+ * The scratch it needs (the longest-first schedule of a packed batch, one
+ * int32 per sequence) lives in a fixed device array inside libgdn.so, sized
+ * for GDN_NOALLOC_MAX_SEQS sequences (16 KiB), which every GPU that loads the
+ * library keeps until the process exits.  It calls no allocator at all.
+ *  - cu_seqlens != NULL with n_seq > GDN_NOALLOC_MAX_SEQS returns
+ *    GDN_ERR_TOO_LARGE and launches nothing (dense batches have no limit).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before capturing a stream into a CUDA graph.
+ *  - All calls share the one array, and every call overwrites the entries it
+ *    uses before reading them, so nothing carries over between calls; but two
+ *    calls that run on the GPU at the same time (different streams, or
+ *    different host threads) race on it and must be serialised by the caller.
+ */
+#define GDN_NOALLOC_MAX_SEQS 4096
+gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, gdn_dtype qkv_dtype,
+                                 const float* g, const float* beta, const float* h0,
+                                 const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int H,
+                                 int K, int V, float scale, void* o, gdn_dtype o_dtype, float* hT,
+                                 unsigned flags, void* stream);
 
 /*
  * gdn_device_status -- reads and clears the device status word on the current
