@@ -58,17 +58,20 @@ constexpr uint32_t OFF_WB = OFF_UB + 8192;       // 2^(G2_L-G2) Ut
 constexpr int AFP = 68;                          // fp32 row pitch of A / T
 constexpr uint32_t OFF_AF = OFF_WB + 8192;
 constexpr uint32_t OFF_TF = OFF_AF + 64 * AFP * 4;
-constexpr int XTP = 20;
+constexpr int XTP = 24;  // pitch of the 16x16 temporaries (conflict-free B fragments)
 constexpr uint32_t OFF_XT = OFF_TF + 64 * AFP * 4;  // fp32 [3][16][20]
 struct Scal {
-    float G2[64];
+    float G2[64];    // in-chunk inclusive cumsum of g, log2 units
     float beta[64];
-    float gam[64];
-    float w[64];
-    float eGL;
+    float gam[64];   // 2^G2
+    float w[64];     // 2^(G2_L - G2)
+    float ginv[64];  // 2^-G2 (only when the chunk's decay stays in fp32 range)
+    float eGL;       // 2^G2_L
     float pad[3];
 };
-constexpr uint32_t OFF_SC = OFF_XT + 3 * 16 * XTP * 4;
+constexpr int OSP = 68;                              // fp32 row pitch of the output stage
+constexpr uint32_t OFF_OS = OFF_XT + 3 * 16 * XTP * 4;   // fp32 [64][68] output rows
+constexpr uint32_t OFF_SC = OFF_OS + 64 * OSP * 4;
 constexpr uint32_t OFF_BAR = OFF_SC + 2 * sizeof(Scal);
 constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
@@ -108,52 +111,57 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t phase, volatile uin
     return false;
 }
 
-// 16x16x16 fp32 product on one warp: acc[2][4] covers rows 2*(lane/4)+{0,1},
-// columns 4*(lane%4)+{0..3}.  Row pitches in floats; Y rows 16-byte aligned.
-__device__ __forceinline__ void mm16(float (&acc)[2][4], const float* X, int xs, const float* Y,
+// 16x16x16 block product on one warp with the warp-level tf32 tensor-core MMA
+// (m16n8k8, fp32 accumulate): C (+)= X Y for fp32 X, Y in shared memory (row
+// pitches in floats).  tcgen05's smallest tile is 64 rows, so the 16x16
+// blocks of the triangular inverse use this form.  Fragment layout (PTX ISA,
+// mma.m16n8k8 .tf32): g = lane/4, t = lane%4; A: (g,t) (g+8,t) (g,t+4)
+// (g+8,t+4); B: (t,g) (t+4,g); C: (g,2t) (g,2t+1) (g+8,2t) (g+8,2t+1).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mm16(float (&c)[2][4], const float* X, int xs, const float* Y,
                                      int ys, int lane) {
-    const int r0 = 2 * (lane >> 2), c0 = 4 * (lane & 3);
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const float a0 = X[r0 * xs + k], a1 = X[(r0 + 1) * xs + k];
-        const float4 y = *reinterpret_cast<const float4*>(Y + k * ys + c0);
-        acc[0][0] = fmaf(a0, y.x, acc[0][0]);
-        acc[0][1] = fmaf(a0, y.y, acc[0][1]);
-        acc[0][2] = fmaf(a0, y.z, acc[0][2]);
-        acc[0][3] = fmaf(a0, y.w, acc[0][3]);
-        acc[1][0] = fmaf(a1, y.x, acc[1][0]);
-        acc[1][1] = fmaf(a1, y.y, acc[1][1]);
-        acc[1][2] = fmaf(a1, y.z, acc[1][2]);
-        acc[1][3] = fmaf(a1, y.w, acc[1][3]);
+    for (int kk = 0; kk < 2; ++kk) {
+        const float* x = X + 8 * kk;
+        uint32_t a[4] = {to_tf32(x[g * xs + t]), to_tf32(x[(g + 8) * xs + t]),
+                         to_tf32(x[g * xs + t + 4]), to_tf32(x[(g + 8) * xs + t + 4])};
+        const float* y = Y + 8 * kk * ys;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+            mma_tf32(c[nt], a, to_tf32(y[t * ys + 8 * nt + g]), to_tf32(y[(t + 4) * ys + 8 * nt + g]));
     }
 }
-__device__ __forceinline__ void mm16_store(const float (&acc)[2][4], float* Z, int zs, int lane,
+__device__ __forceinline__ void mm16_store(const float (&c)[2][4], float* Z, int zs, int lane,
                                            float sign) {
-    const int r0 = 2 * (lane >> 2), c0 = 4 * (lane & 3);
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
-        *reinterpret_cast<float4*>(Z + (r0 + i) * zs + c0) =
-            make_float4(sign * acc[i][0], sign * acc[i][1], sign * acc[i][2], sign * acc[i][3]);
-}
-// Same product restricted to 4 rows (row block rb of 4) on one warp:
-// acc[2] covers row 4*rb + lane/8, columns 2*(lane%8)+{0,1}.
-__device__ __forceinline__ void mm16_rows4(float (&acc)[2], const float* X, int xs, const float* Y,
-                                           int ys, int rb, int lane) {
-    const int r = 4 * rb + (lane >> 3), c0 = 2 * (lane & 7);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const float a = X[r * xs + k];
-        const float2 y = *reinterpret_cast<const float2*>(Y + k * ys + c0);
-        acc[0] = fmaf(a, y.x, acc[0]);
-        acc[1] = fmaf(a, y.y, acc[1]);
+    for (int nt = 0; nt < 2; ++nt) {
+        *reinterpret_cast<float2*>(Z + g * zs + 8 * nt + 2 * t) =
+            make_float2(sign * c[nt][0], sign * c[nt][1]);
+        *reinterpret_cast<float2*>(Z + (g + 8) * zs + 8 * nt + 2 * t) =
+            make_float2(sign * c[nt][2], sign * c[nt][3]);
     }
 }
 
 // T = (I + A)^-1 for the strictly lower 64x64 A (fp32, pitch AFP) by 16x16
-// blocks: diagonal blocks by substitution, then off-diagonal blocks by
-// distance from the diagonal, T_ij = -T_ii sum_{j<=k<i} A_ik T_kj.
-// Writes every T entry on or below the diagonal (diagonal blocks complete).
-// Called by the 128 prep threads; uses named barrier 1.
+// blocks: diagonal blocks by substitution in fp32, then the off-diagonal
+// blocks by distance from the diagonal, T_ij = -T_ii sum_{j<=k<i} A_ik T_kj.
+// Writes every T entry on or below the diagonal (diagonal blocks complete,
+// with their zero upper halves).  Called by the 128 prep threads; uses
+// named barrier 1.
 __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, float* Xt, int pw,
                                                   int lane) {
     // diagonal blocks: warp pw owns block pw, lanes 0..15 one column each
@@ -162,10 +170,13 @@ __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, fl
         float t[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc = fmaf(Af[(o + r) * AFP + o + s], t[s], acc);
-            t[r] = (r < j) ? 0.f : ((r == j) ? 1.f : -acc);
+            for (int s = 0; s < r; s += 2) {
+                acc0 = fmaf(Af[(o + r) * AFP + o + s], t[s], acc0);
+                if (s + 1 < r) acc1 = fmaf(Af[(o + r) * AFP + o + s + 1], t[s + 1], acc1);
+            }
+            t[r] = (r < j) ? 0.f : ((r == j) ? 1.f : -(acc0 + acc1));
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tf[(o + r) * AFP + o + j] = t[r];
@@ -175,43 +186,42 @@ __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, fl
     if (pw < 3) {
         const int i = pw + 1, j = pw;
         float* X = Xt + pw * 16 * XTP;
-        float acc[2][4] = {};
-        mm16(acc, Af + 16 * i * AFP + 16 * j, AFP, Tf + 16 * j * AFP + 16 * j, AFP, lane);
-        mm16_store(acc, X, XTP, lane, 1.f);
+        float c[2][4] = {};
+        mm16(c, Af + 16 * i * AFP + 16 * j, AFP, Tf + 16 * j * AFP + 16 * j, AFP, lane);
+        mm16_store(c, X, XTP, lane, 1.f);
         __syncwarp();
-        float acc2[2][4] = {};
-        mm16(acc2, Tf + 16 * i * AFP + 16 * i, AFP, X, XTP, lane);
-        mm16_store(acc2, Tf + 16 * i * AFP + 16 * j, AFP, lane, -1.f);
+        float c2[2][4] = {};
+        mm16(c2, Tf + 16 * i * AFP + 16 * i, AFP, X, XTP, lane);
+        mm16_store(c2, Tf + 16 * i * AFP + 16 * j, AFP, lane, -1.f);
     }
     tc::named_bar(1, 128);
     // distance 2: blocks (2,0), (3,1)
     if (pw < 2) {
         const int i = pw + 2, j = pw;
         float* X = Xt + pw * 16 * XTP;
-        float acc[2][4] = {};
-        mm16(acc, Af + 16 * i * AFP + 16 * j, AFP, Tf + 16 * j * AFP + 16 * j, AFP, lane);
-        mm16(acc, Af + 16 * i * AFP + 16 * (j + 1), AFP, Tf + 16 * (j + 1) * AFP + 16 * j, AFP,
+        float c[2][4] = {};
+        mm16(c, Af + 16 * i * AFP + 16 * j, AFP, Tf + 16 * j * AFP + 16 * j, AFP, lane);
+        mm16(c, Af + 16 * i * AFP + 16 * (j + 1), AFP, Tf + 16 * (j + 1) * AFP + 16 * j, AFP,
              lane);
-        mm16_store(acc, X, XTP, lane, 1.f);
+        mm16_store(c, X, XTP, lane, 1.f);
         __syncwarp();
-        float acc2[2][4] = {};
-        mm16(acc2, Tf + 16 * i * AFP + 16 * i, AFP, X, XTP, lane);
-        mm16_store(acc2, Tf + 16 * i * AFP + 16 * j, AFP, lane, -1.f);
+        float c2[2][4] = {};
+        mm16(c2, Tf + 16 * i * AFP + 16 * i, AFP, X, XTP, lane);
+        mm16_store(c2, Tf + 16 * i * AFP + 16 * j, AFP, lane, -1.f);
     }
     tc::named_bar(1, 128);
-    // distance 3: block (3,0), rows split over the four warps
-    {
+    // distance 3: block (3,0)
+    if (pw == 0) {
         float* X = Xt;
-        float acc[2] = {0.f, 0.f};
-        mm16_rows4(acc, Af + 48 * AFP + 0, AFP, Tf + 0 * AFP + 0, AFP, pw, lane);
-        mm16_rows4(acc, Af + 48 * AFP + 16, AFP, Tf + 16 * AFP + 0, AFP, pw, lane);
-        mm16_rows4(acc, Af + 48 * AFP + 32, AFP, Tf + 32 * AFP + 0, AFP, pw, lane);
-        const int r = 4 * pw + (lane >> 3), c0 = 2 * (lane & 7);
-        *reinterpret_cast<float2*>(X + r * XTP + c0) = make_float2(acc[0], acc[1]);
-        tc::named_bar(1, 128);
-        float acc2[2] = {0.f, 0.f};
-        mm16_rows4(acc2, Tf + 48 * AFP + 48, AFP, X, XTP, pw, lane);
-        *reinterpret_cast<float2*>(Tf + (48 + r) * AFP + c0) = make_float2(-acc2[0], -acc2[1]);
+        float c[2][4] = {};
+        mm16(c, Af + 48 * AFP + 0, AFP, Tf + 0 * AFP + 0, AFP, lane);
+        mm16(c, Af + 48 * AFP + 16, AFP, Tf + 16 * AFP + 0, AFP, lane);
+        mm16(c, Af + 48 * AFP + 32, AFP, Tf + 32 * AFP + 0, AFP, lane);
+        mm16_store(c, X, XTP, lane, 1.f);
+        __syncwarp();
+        float c2[2][4] = {};
+        mm16(c2, Tf + 48 * AFP + 48, AFP, X, XTP, lane);
+        mm16_store(c2, Tf + 48 * AFP + 0, AFP, lane, -1.f);
     }
     tc::named_bar(1, 128);
 }
@@ -352,9 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             }
             tc::named_bar(1, 128);
             const float G2L = sc->G2[63];
+            // 2^(G2_r - G2_s) = 2^G2_r * 2^-G2_s whenever the chunk's total decay stays
+            // above 2^-126 (no overflow or subnormal factor); else per element
+            const bool factored = G2L > -126.f;
             if (pt < 64) {
                 sc->gam[pt] = exp2f(x);
                 sc->w[pt] = exp2f(G2L - x);
+                sc->ginv[pt] = factored ? exp2f(-x) : 0.f;
             }
             if (pt == 0) sc->eGL = exp2f(G2L);
             // S row of this thread: rows 0-63 = K K^T, rows 64-127 = Q K^T
@@ -369,25 +383,52 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             }
             if (pt == 0) tc::mbar_arrive(&empty[s]);  // stage no longer read by prep
             const uint32_t tp = sbase + OFF_TP + b * SZ_TP;
+            tc::named_bar(1, 128);  // ginv visible
             if (pt < 64) {
                 const int r = pt;
                 const float g2r = sc->G2[r], br = bv;
                 float* arow = Af + r * AFP;
+                if (factored) {
+                    const float coef = br * sc->gam[r];
 #pragma unroll
-                for (int j = 0; j < 64; j += 4) {
-                    float4 av;
-                    av.x = (j + 0 < r) ? br * exp2f(g2r - sc->G2[j + 0]) * sv[j + 0] : 0.f;
-                    av.y = (j + 1 < r) ? br * exp2f(g2r - sc->G2[j + 1]) * sv[j + 1] : 0.f;
-                    av.z = (j + 2 < r) ? br * exp2f(g2r - sc->G2[j + 2]) * sv[j + 2] : 0.f;
-                    av.w = (j + 3 < r) ? br * exp2f(g2r - sc->G2[j + 3]) * sv[j + 3] : 0.f;
-                    *reinterpret_cast<float4*>(arow + j) = av;
+                    for (int j = 0; j < 64; j += 4) {
+                        const float4 gi = *reinterpret_cast<const float4*>(sc->ginv + j);
+                        float4 av;
+                        av.x = (j + 0 < r) ? coef * gi.x * sv[j + 0] : 0.f;
+                        av.y = (j + 1 < r) ? coef * gi.y * sv[j + 1] : 0.f;
+                        av.z = (j + 2 < r) ? coef * gi.z * sv[j + 2] : 0.f;
+                        av.w = (j + 3 < r) ? coef * gi.w * sv[j + 3] : 0.f;
+                        *reinterpret_cast<float4*>(arow + j) = av;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; j += 4) {
+                        float4 av;
+                        av.x = (j + 0 < r) ? br * exp2f(g2r - sc->G2[j + 0]) * sv[j + 0] : 0.f;
+                        av.y = (j + 1 < r) ? br * exp2f(g2r - sc->G2[j + 1]) * sv[j + 1] : 0.f;
+                        av.z = (j + 2 < r) ? br * exp2f(g2r - sc->G2[j + 2]) * sv[j + 2] : 0.f;
+                        av.w = (j + 3 < r) ? br * exp2f(g2r - sc->G2[j + 3]) * sv[j + 3] : 0.f;
+                        *reinterpret_cast<float4*>(arow + j) = av;
+                    }
                 }
             } else {
                 const int r = pt - 64;
                 const float g2r = sc->G2[r];
+                if (factored) {
+                    const float coef = sc->gam[r];
 #pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    sv[j] = (j <= r) ? exp2f(g2r - sc->G2[j]) * sv[j] : 0.f;
+                    for (int j = 0; j < 64; j += 4) {
+                        const float4 gi = *reinterpret_cast<const float4*>(sc->ginv + j);
+                        sv[j + 0] = (j + 0 <= r) ? coef * gi.x * sv[j + 0] : 0.f;
+                        sv[j + 1] = (j + 1 <= r) ? coef * gi.y * sv[j + 1] : 0.f;
+                        sv[j + 2] = (j + 2 <= r) ? coef * gi.z * sv[j + 2] : 0.f;
+                        sv[j + 3] = (j + 3 <= r) ? coef * gi.w * sv[j + 3] : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        sv[j] = (j <= r) ? exp2f(g2r - sc->G2[j]) * sv[j] : 0.f;
+                }
                 tc::store_row_bf16(tp + 8192, r, sv);
             }
             tc::tc_before_sync();
@@ -571,39 +612,53 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 wait(mO, c & 1, abort_flag);
                 tc::tc_after_sync();
                 const float gr = sc->gam[r], scl = p.scale;
+                float* ost = reinterpret_cast<float*>(base + OFF_OS);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float qh[32], pu[32];
                     tc::tmem_ld32(tmem + lane_base + colH + 32 * hf, qh);
                     tc::tmem_ld32(tmem + lane_base + colO + 32 * hf, pu);
                     tc::tmem_wait_ld();
-                    if (r < len) {
-                        const int64_t orow = ((t0 + r) * H + head) * VD + v0 + 32 * hf;
-                        if constexpr (OBF16) {
-                            __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow;
+                    float* orow = ost + r * OSP + 32 * hf;
 #pragma unroll
-                            for (int j = 0; j < 32; j += 8) {
-                                uint4 w4;
-                                w4.x = tc::pack_bf16(scl * fmaf(gr, qh[j], pu[j]),
-                                                     scl * fmaf(gr, qh[j + 1], pu[j + 1]));
-                                w4.y = tc::pack_bf16(scl * fmaf(gr, qh[j + 2], pu[j + 2]),
-                                                     scl * fmaf(gr, qh[j + 3], pu[j + 3]));
-                                w4.z = tc::pack_bf16(scl * fmaf(gr, qh[j + 4], pu[j + 4]),
-                                                     scl * fmaf(gr, qh[j + 5], pu[j + 5]));
-                                w4.w = tc::pack_bf16(scl * fmaf(gr, qh[j + 6], pu[j + 6]),
-                                                     scl * fmaf(gr, qh[j + 7], pu[j + 7]));
-                                *reinterpret_cast<uint4*>(op + j) = w4;
-                            }
-                        } else {
-                            float* op = static_cast<float*>(p.o) + orow;
-#pragma unroll
-                            for (int j = 0; j < 32; j += 4)
-                                *reinterpret_cast<float4*>(op + j) =
-                                    make_float4(scl * fmaf(gr, qh[j], pu[j]),
-                                                scl * fmaf(gr, qh[j + 1], pu[j + 1]),
-                                                scl * fmaf(gr, qh[j + 2], pu[j + 2]),
-                                                scl * fmaf(gr, qh[j + 3], pu[j + 3]));
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(orow + j) =
+                            make_float4(scl * fmaf(gr, qh[j], pu[j]),
+                                        scl * fmaf(gr, qh[j + 1], pu[j + 1]),
+                                        scl * fmaf(gr, qh[j + 2], pu[j + 2]),
+                                        scl * fmaf(gr, qh[j + 3], pu[j + 3]));
+                }
+                tc::named_bar(3, 64);
+                // coalesced stores: consecutive threads cover consecutive 16-byte
+                // pieces of one output row
+                const int ot = ct - 64;
+                if constexpr (OBF16) {
+                    __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.o);
+#pragma unroll 2
+                    for (int it = 0; it < 8; ++it) {
+                        const int rr = 8 * it + (ot >> 3), c8 = 8 * (ot & 7);
+                        if (rr < len) {
+                            const float4 a = *reinterpret_cast<const float4*>(ost + rr * OSP + c8);
+                            const float4 bq =
+                                *reinterpret_cast<const float4*>(ost + rr * OSP + c8 + 4);
+                            uint4 w4;
+                            w4.x = tc::pack_bf16(a.x, a.y);
+                            w4.y = tc::pack_bf16(a.z, a.w);
+                            w4.z = tc::pack_bf16(bq.x, bq.y);
+                            w4.w = tc::pack_bf16(bq.z, bq.w);
+                            *reinterpret_cast<uint4*>(obase + ((t0 + rr) * H + head) * VD + v0 +
+                                                      c8) = w4;
                         }
+                    }
+                } else {
+                    float* obase = static_cast<float*>(p.o);
+#pragma unroll 4
+                    for (int it = 0; it < 16; ++it) {
+                        const int rr = 4 * it + (ot >> 4), c4 = 4 * (ot & 15);
+                        if (rr < len)
+                            *reinterpret_cast<float4*>(obase + ((t0 + rr) * H + head) * VD + v0 +
+                                                       c4) =
+                                *reinterpret_cast<const float4*>(ost + rr * OSP + c4);
                     }
                 }
                 tc::tc_before_sync();
