@@ -179,6 +179,8 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int, dev) -> float:
+    """Max of a per-rank scalar over the process group (nccl: dev is the rank's
+    GPU; gloo: a CPU device)."""
     if world == 1:
         return x
     import torch.distributed as dist
