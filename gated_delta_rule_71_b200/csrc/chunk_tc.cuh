@@ -1,28 +1,35 @@
 // chunk_tc.cuh -- fused tensor-core chunked forward of the gated delta rule
 // (bf16 q/k/v, K = V = 128, fp32 state, fp32 accumulation), sm_100a.
 //
-// One CTA owns one (sequence, head, 64-wide value slice) and walks its chunks
-// in order; the three steps of ZzCompute (PyTorch Helion Hackathon gallery
-// entry 11) -- item 4 "Recompute W/U" (in-chunk cumsum, A, T = (I+A)^-1),
-// item 2 "Chunk Forward H" (state recurrence) and item 3 "Chunk Forward O"
-// (chunk output) -- run in one kernel so q/k/v/g/beta are read from HBM once and
-// o/h_T written once.  Per chunk (64 tokens, G2 = log2-scaled cumsum of g):
+// The three GDN steps of ZzCompute (PyTorch Helion Hackathon gallery entry 11)
+// -- item 4 "Recompute W/U" (in-chunk cumsum, A, T = (I+A)^-1), item 2 "Chunk
+// Forward H" (state recurrence) and item 3 "Chunk Forward O" (chunk output) --
+// run in one launch, so q/k/v/g/beta are read from HBM once and o/h_T written
+// once.  Per chunk (64 tokens, G2 = log2-scaled in-chunk cumsum of g):
 //   S    = [K; Q] K^T                               (MMA, M=128 N=64 K=128)
-//   A    = strictly-lower beta_r 2^(G2_r-G2_s) (K K^T)_rs,  T = (I + A)^-1 (SIMT fp32)
-//   P    = lower-incl 2^(G2_r-G2_s) (Q K^T)_rs                              (SIMT)
+//   A    = strictly-lower beta_r 2^(G2_r-G2_s) (K K^T)_rs,  T = (I + A)^-1
+//   P    = lower-incl 2^(G2_r-G2_s) (Q K^T)_rs
 //   [KH; QH] = [K; Q] h                             (MMA, B = bf16 copy of h)
-//   R    = beta (V - 2^G2 * KH)                                        (SIMT)
+//   R    = beta (V - 2^G2 * KH)
 //   Ut   = T R             ( = U - W h of the WY form)  (MMA, A = [T; P])
 //   h'   = 2^G2_L h + K^T (2^(G2_L-G2) * Ut)            (MMA, then fp32 update)
 //   O    = scale (2^G2 * QH + P Ut)                      (MMA, A = [T; P])
-// Warp roles (384 threads): warp 0 issues TMA loads into a 2-stage ring and
-// owns tensor memory; warps 4-7 ("prep") build A, T and P for each chunk one
-// chunk ahead; warps 8-11 ("chain") carry the fp32 state in registers through
-// the serial part and write the output.  Every MMA is issued by one thread of
-// the warpgroup that consumes it, with completion signalled on an mbarrier.
-// Every wait is bounded: a wait that gives up sets an abort flag (all later
-// waits fall through, so every named barrier is still reached) and records
-// GDN_ERR_TIMEOUT in the device status word.
+//
+// Each (sequence, head) runs on a cluster of two CTAs, one per SM:
+//  * rank 0, "prep": three warpgroups, each owning every third chunk, its own
+//    TMA stage and its own slot in the chain CTA.  A warpgroup computes S on
+//    tcgen05, the A and P rows, and T by 16x16 blocks, and writes T, P (bf16)
+//    and the per-row gate factors straight into the chain CTA's shared memory
+//    (DSMEM), then releases them with cluster-scope mbarrier arrives.  Three
+//    chunks are in flight, so the serial triangular inverse is off the chain.
+//  * rank 1, "chain": four warpgroups, one per 32 value columns, carry the
+//    fp32 state in registers (one key row per thread) through the serial part
+//    with N = 128 tcgen05 MMAs and write the output rows.
+// TMA loads are issued by the thread that releases a stage, so no producer
+// warp waits.  Every wait is bounded: a wait that gives up sets the CTA's
+// abort flag (all later waits fall through, so every barrier is still
+// reached), records GDN_ERR_TIMEOUT, and the issuing threads drain their
+// copies and MMAs before tensor memory is released.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -39,53 +46,79 @@ namespace tcf {
 constexpr int C = 64;    // chunk
 constexpr int KD = 128;  // key dim
 constexpr int VD = 128;  // value dim
-constexpr int VS = 64;   // value slice per CTA
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int NPREP = 3;  // prep warpgroups (chunks in flight in the prep CTA)
 constexpr uint32_t kPolls = 1u << 22;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// shared memory (byte offsets from a 1024-aligned base)
+// ---- shared memory, prep CTA (byte offsets from a 1024-aligned base)
 constexpr uint32_t SZ_KQ = 32768;  // [2 key halves][K rows 0-63 | Q rows 64-127][128 B]
-constexpr uint32_t SZ_V = 8192;    // [64 rows][64 bf16]
+constexpr int AFP = 68;            // fp32 row pitch of A / T
+constexpr int XTP = 24;            // pitch of the 16x16 temporaries (conflict-free B fragments)
+constexpr uint32_t SZ_AF = 64 * AFP * 4;
+constexpr uint32_t SZ_XT = 3 * 16 * XTP * 4;
+struct PrepScal {   // per prep warpgroup
+    float G2[64];   // in-chunk inclusive cumsum of g, log2 units
+    float ginv[64]; // 2^-G2 (only when the chunk's decay stays in fp32 range)
+    float gam[64];  // 2^G2
+    float pad;
+    float scan_tmp;
+    float pad2[2];
+};
+constexpr uint32_t P_OFF_KQ = 0;                                  // NPREP stages
+constexpr uint32_t P_OFF_AF = P_OFF_KQ + NPREP * SZ_KQ;           // NPREP x A
+constexpr uint32_t P_OFF_TF = P_OFF_AF + NPREP * SZ_AF;           // NPREP x T
+constexpr uint32_t P_OFF_XT = P_OFF_TF + NPREP * SZ_AF;           // NPREP x temporaries
+constexpr uint32_t P_OFF_SC = P_OFF_XT + NPREP * SZ_XT;           // NPREP x PrepScal
+constexpr uint32_t P_END = P_OFF_SC + NPREP * sizeof(PrepScal);
+
+// ---- shared memory, chain CTA
+constexpr uint32_t SZ_V = 16384;   // [2 atoms of 64 v][64 rows][128 B]
 constexpr uint32_t SZ_TP = 16384;  // [T rows 0-63 | P rows 64-127][64 bf16]
-constexpr uint32_t OFF_KQ = 0;
-constexpr uint32_t OFF_V = OFF_KQ + 2 * SZ_KQ;
-constexpr uint32_t OFF_TP = OFF_V + 2 * SZ_V;
-constexpr uint32_t OFF_HB = OFF_TP + 2 * SZ_TP;  // h bf16 [128 key rows][64 v]
-constexpr uint32_t OFF_RB = OFF_HB + 16384;      // R  [64 rows][64 v]
-constexpr uint32_t OFF_UB = OFF_RB + 8192;       // Ut
-constexpr uint32_t OFF_WB = OFF_UB + 8192;       // 2^(G2_L-G2) Ut
-constexpr int AFP = 68;                          // fp32 row pitch of A / T
-constexpr uint32_t OFF_AF = OFF_WB + 8192;
-constexpr uint32_t OFF_TF = OFF_AF + 64 * AFP * 4;
-constexpr int XTP = 24;  // pitch of the 16x16 temporaries (conflict-free B fragments)
-constexpr uint32_t OFF_XT = OFF_TF + 64 * AFP * 4;  // fp32 [3][16][20]
-struct Scal {
-    float G2[64];    // in-chunk inclusive cumsum of g, log2 units
+struct ChainScal {  // per slot, written by the prep CTA
     float beta[64];
-    float gam[64];   // 2^G2
-    float w[64];     // 2^(G2_L - G2)
-    float ginv[64];  // 2^-G2 (only when the chunk's decay stays in fp32 range)
-    float eGL;       // 2^G2_L
+    float gam[64];  // 2^G2
+    float w[64];    // 2^(G2_L - G2)
+    float eGL;      // 2^G2_L
     float pad[3];
 };
-constexpr int OSP = 68;                              // fp32 row pitch of the output stage
-constexpr uint32_t OFF_OS = OFF_XT + 3 * 16 * XTP * 4;   // fp32 [64][68] output rows
-constexpr uint32_t OFF_SC = OFF_OS + 64 * OSP * 4;
-constexpr uint32_t OFF_BAR = OFF_SC + 2 * sizeof(Scal);
-constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
+constexpr uint32_t C_OFF_KQ = 0;                                // 2 stages
+constexpr uint32_t C_OFF_V = C_OFF_KQ + 2 * SZ_KQ;              // 1 buffer (refilled after R)
+constexpr uint32_t C_OFF_TP = C_OFF_V + SZ_V;                   // NPREP slots
+constexpr uint32_t C_OFF_HB = C_OFF_TP + NPREP * SZ_TP;         // h bf16 [2 atoms][128][128 B]
+constexpr uint32_t C_OFF_RB = C_OFF_HB + 32768;                 // R [2 atoms][64][128 B]
+constexpr uint32_t C_OFF_UB = C_OFF_RB + 16384;                 // Ut
+constexpr uint32_t C_OFF_WB = C_OFF_UB + 16384;                 // 2^(G2_L-G2) Ut
+constexpr uint32_t C_OFF_OS = C_OFF_UB;                         // fp32 output rows [64][128]
+constexpr uint32_t C_OFF_SC = C_OFF_WB + 16384;                 // NPREP x ChainScal
+constexpr uint32_t C_END = C_OFF_SC + NPREP * sizeof(ChainScal);
 
-// tensor memory columns (fp32 accumulators, 128 lanes each)
-constexpr uint32_t COL_S = 0;
-constexpr uint32_t COL_H = 64;   // two buffers
-constexpr uint32_t COL_U = 192;
-constexpr uint32_t COL_D = 256;
-constexpr uint32_t COL_O = 320;  // two buffers
-constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t BODY = (P_END > C_END ? P_END : C_END);
+constexpr uint32_t OFF_BAR = (BODY + 15) & ~15u;
+constexpr uint32_t OFF_MISC = OFF_BAR + 32 * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// ---- tensor memory columns
+constexpr uint32_t P_COL_S = 0;  // NPREP x 64 in the prep CTA
+constexpr uint32_t P_TMEM_COLS = 256;
+constexpr uint32_t C_COL_H = 0;    // two buffers of 128
+constexpr uint32_t C_COL_U = 256;  // Ut, then [T Ut; P Ut]
+constexpr uint32_t C_COL_D = 384;  // K^T (w Ut)
+constexpr uint32_t C_TMEM_COLS = 512;
+
+// barrier slots
+enum : int {
+    B_FULL = 0,        // [NPREP] prep: TMA stage; chain uses [0..1]
+    B_MS = 3,          // [NPREP] prep: S ready
+    B_FREE = 6,        // [NPREP] prep: chain slot free (remote arrivals)
+    B_TPF = 9,         // [NPREP] chain: slot filled (remote arrivals, 128 each)
+    B_MH = 12, B_MU, B_MD, B_MO, B_DRAIN,
+    B_FULLV,           // chain: V tile
+};
 
 struct Params {
-    CUtensorMap tm_q, tm_k, tm_v;
+    CUtensorMap tm_q, tm_k, tm_v, tm_o;  // tm_o: fp32 output, 32 x 64 boxes
     const float* g;
     const float* beta;
     const float* h0;
@@ -98,17 +131,26 @@ struct Params {
     float* hT;
 };
 
-// Bounded wait that honours the block's abort flag.
-__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t phase, volatile uint32_t* abort) {
+// Bounded wait that honours the CTA's abort flag.  `cluster` selects
+// acquire at cluster scope (arrivals from the other CTA).
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t phase, volatile uint32_t* abort,
+                                     bool cluster = false) {
     if (*abort) return false;
     const uint32_t a = smem_u32(bar);
     for (uint32_t i = 0; i < kPolls; ++i) {
-        if (mbar_try_wait(a, phase)) return true;
+        if (cluster ? tc::mbar_try_wait_cluster(a, phase) : mbar_try_wait(a, phase)) return true;
         if ((i & 255u) == 255u && *abort) return false;
     }
     *abort = 1u;
     record_status(GDN_ERR_TIMEOUT);
     return false;
+}
+
+// Bounded wait that ignores the abort flag (used to drain on the way out).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t phase) {
+    const uint32_t a = smem_u32(bar);
+    for (uint32_t i = 0; i < kPolls && !mbar_try_wait(a, phase); ++i) {
+    }
 }
 
 // 16x16x16 block product on one warp with the warp-level tf32 tensor-core MMA
@@ -160,10 +202,10 @@ __device__ __forceinline__ void mm16_store(const float (&c)[2][4], float* Z, int
 // blocks: diagonal blocks by substitution in fp32, then the off-diagonal
 // blocks by distance from the diagonal, T_ij = -T_ii sum_{j<=k<i} A_ik T_kj.
 // Writes every T entry on or below the diagonal (diagonal blocks complete,
-// with their zero upper halves).  Called by the 128 prep threads; uses
-// named barrier 1.
+// with their zero upper halves).  Called by the 128 threads of one prep
+// warpgroup; uses named barrier `bid`.
 __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, float* Xt, int pw,
-                                                  int lane) {
+                                                  int lane, int bid) {
     // diagonal blocks: warp pw owns block pw, lanes 0..15 one column each
     if (lane < 16) {
         const int o = 16 * pw, j = lane;
@@ -181,7 +223,7 @@ __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, fl
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tf[(o + r) * AFP + o + j] = t[r];
     }
-    tc::named_bar(1, 128);
+    tc::named_bar(bid, 128);
     // distance 1: blocks (1,0), (2,1), (3,2)
     if (pw < 3) {
         const int i = pw + 1, j = pw;
@@ -194,7 +236,7 @@ __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, fl
         mm16(c2, Tf + 16 * i * AFP + 16 * i, AFP, X, XTP, lane);
         mm16_store(c2, Tf + 16 * i * AFP + 16 * j, AFP, lane, -1.f);
     }
-    tc::named_bar(1, 128);
+    tc::named_bar(bid, 128);
     // distance 2: blocks (2,0), (3,1)
     if (pw < 2) {
         const int i = pw + 2, j = pw;
@@ -209,7 +251,7 @@ __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, fl
         mm16(c2, Tf + 16 * i * AFP + 16 * i, AFP, X, XTP, lane);
         mm16_store(c2, Tf + 16 * i * AFP + 16 * j, AFP, lane, -1.f);
     }
-    tc::named_bar(1, 128);
+    tc::named_bar(bid, 128);
     // distance 3: block (3,0)
     if (pw == 0) {
         float* X = Xt;
@@ -223,8 +265,9 @@ __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, fl
         mm16(c2, Tf + 48 * AFP + 48, AFP, X, XTP, lane);
         mm16_store(c2, Tf + 48 * AFP + 0, AFP, lane, -1.f);
     }
-    tc::named_bar(1, 128);
+    tc::named_bar(bid, 128);
 }
+
 
 template <bool OBF16>
 __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_constant__ Params p) {
@@ -234,25 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
     uint8_t* base = smem_raw + (sbase - raw_u32);
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + OFF_BAR);
-    uint64_t* full = bars + 0;
-    uint64_t* empty = bars + 2;
-    uint64_t* pfull = bars + 4;
-    uint64_t* pempty = bars + 6;
-    uint64_t* mS = bars + 8;
-    uint64_t* mH = bars + 9;
-    uint64_t* mU = bars + 10;
-    uint64_t* mD = bars + 11;
-    uint64_t* mO = bars + 12;
-    uint64_t* mDrain = bars + 13;   // chain-side drain after an abort
-    uint64_t* mDrainP = bars + 14;  // prep-side drain after an abort
     uint32_t* misc = reinterpret_cast<uint32_t*>(base + OFF_MISC);
     volatile uint32_t* abort_flag = misc + 1;
-    float* scan_tmp = reinterpret_cast<float*>(misc + 2);
-    Scal* SC = reinterpret_cast<Scal*>(base + OFF_SC);
 
+    const uint32_t rank = tc::cluster_ctarank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = p.H;
-    const int vsl = blockIdx.x & 1;
     const int sh = blockIdx.x >> 1;
     const int head = sh % H;
     const int slot = sh / H;
@@ -266,325 +296,355 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
         ce = cs + p.T;
     }
     const int nch = (int)((ce - cs + C - 1) / C);
-    const int v0 = vsl * VS;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 2);
-            mbar_init(&pfull[i], 1);
-            mbar_init(&pempty[i], 64);
-        }
-        mbar_init(mS, 1);
-        mbar_init(mH, 1);
-        mbar_init(mU, 1);
-        mbar_init(mD, 1);
-        mbar_init(mO, 1);
-        mbar_init(mDrain, 1);
-        mbar_init(mDrainP, 1);
+        for (int i = 0; i < 32; ++i)
+            mbar_init(&bars[i], (i >= B_TPF && i < B_TPF + NPREP) ? 128u : 1u);
         misc[1] = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) tc::tmem_alloc(&misc[0], TMEM_COLS);
+    const uint32_t ncols = rank == 0 ? P_TMEM_COLS : C_TMEM_COLS;
+    if (warp == 0) tc::tmem_alloc(&misc[0], ncols);
     tc::tc_before_sync();
     __syncthreads();
+    tc::cluster_sync();  // both CTAs' barriers initialised before any remote arrive
     tc::tc_after_sync();
     const uint32_t tmem = misc[0];
 
-    if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tc::prefetch_tmap(&p.tm_q);
-            tc::prefetch_tmap(&p.tm_k);
-            tc::prefetch_tmap(&p.tm_v);
-            for (int c = 0; c < nch; ++c) {
-                const int s = c & 1;
-                if (c >= 2) wait(&empty[s], ((c >> 1) + 1) & 1, abort_flag);
-                tc::mbar_arrive_expect_tx(&full[s], SZ_KQ + SZ_V);
+    if (rank == 0) {
+        // ================================================================ prep
+        const int wg = warp >> 2;  // 0..3; warpgroups 1..NPREP work
+        if (wg >= 1 && wg <= NPREP) {
+            const int pg = wg - 1, pt = threadIdx.x - 128 * wg, pw = warp & 3;
+            const int bid = 1 + pg;
+            uint8_t* kq_p = base + P_OFF_KQ + pg * SZ_KQ;
+            const uint32_t kq = sbase + P_OFF_KQ + pg * SZ_KQ;
+            float* Af = reinterpret_cast<float*>(base + P_OFF_AF + pg * SZ_AF);
+            float* Tf = reinterpret_cast<float*>(base + P_OFF_TF + pg * SZ_AF);
+            float* Xt = reinterpret_cast<float*>(base + P_OFF_XT + pg * SZ_XT);
+            PrepScal* ls = reinterpret_cast<PrepScal*>(base + P_OFF_SC) + pg;
+            uint64_t* full = &bars[B_FULL + pg];
+            uint64_t* mS = &bars[B_MS + pg];
+            uint64_t* sfree = &bars[B_FREE + pg];
+            // the chain CTA's slot for this warpgroup
+            const uint32_t r_tp = tc::mapa(sbase + C_OFF_TP + pg * SZ_TP, 1);
+            const uint32_t r_sc = tc::mapa(sbase + C_OFF_SC + pg * (uint32_t)sizeof(ChainScal), 1);
+            const uint32_t r_tpf = tc::mapa(smem_u32(&bars[B_TPF + pg]), 1);
+            const uint32_t idS = tc::idesc_bf16(128, 64, 0, 0);
+            auto issue_load = [&](int c) {
                 const int y = (int)(cs + (int64_t)C * c);
-                uint8_t* kq = base + OFF_KQ + s * SZ_KQ;
-                tc::tma_load_2d(kq + 0, &p.tm_k, head * KD + 0, y, &full[s]);
-                tc::tma_load_2d(kq + 8192, &p.tm_q, head * KD + 0, y, &full[s]);
-                tc::tma_load_2d(kq + 16384, &p.tm_k, head * KD + 64, y, &full[s]);
-                tc::tma_load_2d(kq + 24576, &p.tm_q, head * KD + 64, y, &full[s]);
-                tc::tma_load_2d(base + OFF_V + s * SZ_V, &p.tm_v, head * VD + v0, y, &full[s]);
+                tc::mbar_arrive_expect_tx(full, SZ_KQ);
+                tc::tma_load_2d(kq_p + 0, &p.tm_k, head * KD + 0, y, full);
+                tc::tma_load_2d(kq_p + 8192, &p.tm_q, head * KD + 0, y, full);
+                tc::tma_load_2d(kq_p + 16384, &p.tm_k, head * KD + 64, y, full);
+                tc::tma_load_2d(kq_p + 24576, &p.tm_q, head * KD + 64, y, full);
+            };
+            int last_loaded = -1;
+            if (pt == 0 && pg < nch) {
+                tc::prefetch_tmap(&p.tm_q);
+                tc::prefetch_tmap(&p.tm_k);
+                issue_load(pg);
+                last_loaded = pg;
             }
-            // never leave with copies in flight
-            for (int c = (nch > 2 ? nch - 2 : 0); c < nch; ++c) {
-                const uint32_t a = smem_u32(&full[c & 1]);
-                for (uint32_t i = 0; i < kPolls && !mbar_try_wait(a, (c >> 1) & 1); ++i) {
+            for (int c = pg, n = 0; c < nch; c += NPREP, ++n) {
+                const int64_t t0 = cs + (int64_t)C * c;
+                const int len = (int)((ce - t0) < C ? (ce - t0) : C);
+                float gv = 0.f, bv = 0.f;
+                if (pt < len) {
+                    gv = p.g[(t0 + pt) * H + head];
+                    bv = p.beta[(t0 + pt) * H + head];
                 }
-            }
-        }
-    } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------------------------- prep
-        const int pt = threadIdx.x - 128, pw = warp - 4;
-        float* Af = reinterpret_cast<float*>(base + OFF_AF);
-        float* Tf = reinterpret_cast<float*>(base + OFF_TF);
-        float* Xt = reinterpret_cast<float*>(base + OFF_XT);
-        const uint32_t idS = tc::idesc_bf16(128, 64, 0, 0);
-        for (int c = 0; c < nch; ++c) {
-            const int s = c & 1, b = c & 1;
-            const int64_t t0 = cs + (int64_t)C * c;
-            const int len = (int)((ce - t0) < C ? (ce - t0) : C);
-            float gv = 0.f, bv = 0.f;
-            if (pt < len) {
-                gv = p.g[(t0 + pt) * H + head];
-                bv = p.beta[(t0 + pt) * H + head];
-            }
-            wait(&full[s], (c >> 1) & 1, abort_flag);
-            const uint32_t kq = sbase + OFF_KQ + s * SZ_KQ;
-            if (pt == 0) {
+                wait(full, n & 1, abort_flag);
+                if (pt == 0) {
+                    tc::tc_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        tc::mma_bf16(tmem + P_COL_S + 64 * pg, tc::sdesc_sw128(kq + off, 16, 1024),
+                                     tc::sdesc_sw128(kq + off, 16, 1024), idS, kk > 0);
+                    }
+                    tc::mma_commit(mS);
+                }
+                // in-chunk inclusive cumsum of g (log2 units) on warps 0-1
+                float x = gv * kLog2e;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                if (pt == 31) ls->scan_tmp = x;
+                if (n >= 1) wait(sfree, (n - 1) & 1, abort_flag, true);  // chain done with the slot
+                tc::named_bar(bid, 128);
+                if (pw == 1) x += ls->scan_tmp;
+                if (pt < 64) ls->G2[pt] = x;
+                tc::named_bar(bid, 128);
+                const float G2L = ls->G2[63];
+                // 2^(G2_r - G2_s) = 2^G2_r * 2^-G2_s whenever the chunk's total decay
+                // stays above 2^-126 (no overflow or subnormal factor); else per element
+                const bool factored = G2L > -126.f;
+                if (pt < 64) {
+                    const float gm = exp2f(x);
+                    ls->gam[pt] = gm;
+                    ls->ginv[pt] = factored ? exp2f(-x) : 0.f;
+                    tc::st_cluster_f32(r_sc + 4 * (0 * 64 + pt), bv);
+                    tc::st_cluster_f32(r_sc + 4 * (1 * 64 + pt), gm);
+                    tc::st_cluster_f32(r_sc + 4 * (2 * 64 + pt), exp2f(G2L - x));
+                    if (pt == 0) tc::st_cluster_f32(r_sc + 4 * (3 * 64), exp2f(G2L));
+                }
+                // S row of this thread: rows 0-63 = K K^T, rows 64-127 = Q K^T
+                wait(mS, n & 1, abort_flag);
                 tc::tc_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    tc::mma_bf16(tmem + COL_S, tc::sdesc_sw128(kq + off, 16, 1024),
-                                 tc::sdesc_sw128(kq + off, 16, 1024), idS, kk > 0);
+                float sv[64];
+                {
+                    const uint32_t ta = tmem + ((uint32_t)(32 * pw) << 16) + P_COL_S + 64 * pg;
+                    tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(sv));
+                    tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+                    tc::tmem_wait_ld();
                 }
-                tc::mma_commit(mS);
-            }
-            // in-chunk inclusive cumsum of g (log2 units) on warps 0-1
-            float x = gv * kLog2e;
+                // the stage is no longer read: fetch this warpgroup's next chunk into it
+                if (pt == 0 && c + NPREP < nch) {
+                    issue_load(c + NPREP);
+                    last_loaded = c + NPREP;
+                }
+                tc::named_bar(bid, 128);  // ginv / gam visible
+                if (pt < 64) {
+                    const int r = pt;
+                    const float g2r = ls->G2[r], br = bv;
+                    float* arow = Af + r * AFP;
+                    if (factored) {
+                        const float coef = br * ls->gam[r];
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, off);
-                if (lane >= off) x += y;
-            }
-            if (pt == 31) *scan_tmp = x;
-            if (c >= 2) wait(&pempty[b], ((c >> 1) + 1) & 1, abort_flag);
-            tc::named_bar(1, 128);
-            if (pw == 1) x += *scan_tmp;
-            Scal* sc = SC + b;
-            if (pt < 64) {
-                sc->G2[pt] = x;
-                sc->beta[pt] = bv;
-            }
-            tc::named_bar(1, 128);
-            const float G2L = sc->G2[63];
-            // 2^(G2_r - G2_s) = 2^G2_r * 2^-G2_s whenever the chunk's total decay stays
-            // above 2^-126 (no overflow or subnormal factor); else per element
-            const bool factored = G2L > -126.f;
-            if (pt < 64) {
-                sc->gam[pt] = exp2f(x);
-                sc->w[pt] = exp2f(G2L - x);
-                sc->ginv[pt] = factored ? exp2f(-x) : 0.f;
-            }
-            if (pt == 0) sc->eGL = exp2f(G2L);
-            // S row of this thread: rows 0-63 = K K^T, rows 64-127 = Q K^T
-            wait(mS, c & 1, abort_flag);
-            tc::tc_after_sync();
-            float sv[64];
-            {
-                const uint32_t ta = tmem + ((uint32_t)(32 * pw) << 16) + COL_S;
-                tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(sv));
-                tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
-                tc::tmem_wait_ld();
-            }
-            if (pt == 0) tc::mbar_arrive(&empty[s]);  // stage no longer read by prep
-            const uint32_t tp = sbase + OFF_TP + b * SZ_TP;
-            tc::named_bar(1, 128);  // ginv visible
-            if (pt < 64) {
-                const int r = pt;
-                const float g2r = sc->G2[r], br = bv;
-                float* arow = Af + r * AFP;
-                if (factored) {
-                    const float coef = br * sc->gam[r];
+                        for (int j = 0; j < 64; j += 4) {
+                            const float4 gi = *reinterpret_cast<const float4*>(ls->ginv + j);
+                            float4 av;
+                            av.x = (j + 0 < r) ? coef * gi.x * sv[j + 0] : 0.f;
+                            av.y = (j + 1 < r) ? coef * gi.y * sv[j + 1] : 0.f;
+                            av.z = (j + 2 < r) ? coef * gi.z * sv[j + 2] : 0.f;
+                            av.w = (j + 3 < r) ? coef * gi.w * sv[j + 3] : 0.f;
+                            *reinterpret_cast<float4*>(arow + j) = av;
+                        }
+                    } else {
 #pragma unroll
-                    for (int j = 0; j < 64; j += 4) {
-                        const float4 gi = *reinterpret_cast<const float4*>(sc->ginv + j);
-                        float4 av;
-                        av.x = (j + 0 < r) ? coef * gi.x * sv[j + 0] : 0.f;
-                        av.y = (j + 1 < r) ? coef * gi.y * sv[j + 1] : 0.f;
-                        av.z = (j + 2 < r) ? coef * gi.z * sv[j + 2] : 0.f;
-                        av.w = (j + 3 < r) ? coef * gi.w * sv[j + 3] : 0.f;
-                        *reinterpret_cast<float4*>(arow + j) = av;
+                        for (int j = 0; j < 64; j += 4) {
+                            float4 av;
+                            av.x = (j + 0 < r) ? br * exp2f(g2r - ls->G2[j + 0]) * sv[j + 0] : 0.f;
+                            av.y = (j + 1 < r) ? br * exp2f(g2r - ls->G2[j + 1]) * sv[j + 1] : 0.f;
+                            av.z = (j + 2 < r) ? br * exp2f(g2r - ls->G2[j + 2]) * sv[j + 2] : 0.f;
+                            av.w = (j + 3 < r) ? br * exp2f(g2r - ls->G2[j + 3]) * sv[j + 3] : 0.f;
+                            *reinterpret_cast<float4*>(arow + j) = av;
+                        }
                     }
                 } else {
+                    const int r = pt - 64;
+                    const float g2r = ls->G2[r];
+                    if (factored) {
+                        const float coef = ls->gam[r];
 #pragma unroll
-                    for (int j = 0; j < 64; j += 4) {
-                        float4 av;
-                        av.x = (j + 0 < r) ? br * exp2f(g2r - sc->G2[j + 0]) * sv[j + 0] : 0.f;
-                        av.y = (j + 1 < r) ? br * exp2f(g2r - sc->G2[j + 1]) * sv[j + 1] : 0.f;
-                        av.z = (j + 2 < r) ? br * exp2f(g2r - sc->G2[j + 2]) * sv[j + 2] : 0.f;
-                        av.w = (j + 3 < r) ? br * exp2f(g2r - sc->G2[j + 3]) * sv[j + 3] : 0.f;
-                        *reinterpret_cast<float4*>(arow + j) = av;
+                        for (int j = 0; j < 64; j += 4) {
+                            const float4 gi = *reinterpret_cast<const float4*>(ls->ginv + j);
+                            sv[j + 0] = (j + 0 <= r) ? coef * gi.x * sv[j + 0] : 0.f;
+                            sv[j + 1] = (j + 1 <= r) ? coef * gi.y * sv[j + 1] : 0.f;
+                            sv[j + 2] = (j + 2 <= r) ? coef * gi.z * sv[j + 2] : 0.f;
+                            sv[j + 3] = (j + 3 <= r) ? coef * gi.w * sv[j + 3] : 0.f;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j)
+                            sv[j] = (j <= r) ? exp2f(g2r - ls->G2[j]) * sv[j] : 0.f;
+                    }
+                    // P row -> the chain CTA's slot (rows 64-127 of the stacked operand)
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        tc::st_cluster_v4(r_tp + 8192 + tc::sw128_off(r, ch),
+                                          tc::pack_bf16(sv[8 * ch + 0], sv[8 * ch + 1]),
+                                          tc::pack_bf16(sv[8 * ch + 2], sv[8 * ch + 3]),
+                                          tc::pack_bf16(sv[8 * ch + 4], sv[8 * ch + 5]),
+                                          tc::pack_bf16(sv[8 * ch + 6], sv[8 * ch + 7]));
+                }
+                tc::tc_before_sync();
+                tc::named_bar(bid, 128);
+                invert_unit_lower(Af, Tf, Xt, pw, lane, bid);
+                {
+                    // T rows -> bf16 (upper part zero) into the chain CTA's slot
+                    const int r = pt >> 1, hf = pt & 1;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int ch = 4 * hf + q4;
+                        float t8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int col = 8 * ch + e;
+                            t8[e] = (col <= r) ? Tf[r * AFP + col] : 0.f;
+                        }
+                        tc::st_cluster_v4(r_tp + tc::sw128_off(r, ch), tc::pack_bf16(t8[0], t8[1]),
+                                          tc::pack_bf16(t8[2], t8[3]), tc::pack_bf16(t8[4], t8[5]),
+                                          tc::pack_bf16(t8[6], t8[7]));
                     }
                 }
-            } else {
-                const int r = pt - 64;
-                const float g2r = sc->G2[r];
-                if (factored) {
-                    const float coef = sc->gam[r];
-#pragma unroll
-                    for (int j = 0; j < 64; j += 4) {
-                        const float4 gi = *reinterpret_cast<const float4*>(sc->ginv + j);
-                        sv[j + 0] = (j + 0 <= r) ? coef * gi.x * sv[j + 0] : 0.f;
-                        sv[j + 1] = (j + 1 <= r) ? coef * gi.y * sv[j + 1] : 0.f;
-                        sv[j + 2] = (j + 2 <= r) ? coef * gi.z * sv[j + 2] : 0.f;
-                        sv[j + 3] = (j + 3 <= r) ? coef * gi.w * sv[j + 3] : 0.f;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        sv[j] = (j <= r) ? exp2f(g2r - sc->G2[j]) * sv[j] : 0.f;
-                }
-                tc::store_row_bf16(tp + 8192, r, sv);
+                // publish: the chain CTA's MMAs read the slot through the async proxy
+                tc::fence_async_cluster();
+                tc::mbar_arrive_cluster(r_tpf);
             }
-            tc::tc_before_sync();
-            tc::named_bar(1, 128);
-            invert_unit_lower(Af, Tf, Xt, pw, lane);
-            {
-                // T rows -> bf16 (upper part zero), two threads per row
-                const int r = pt >> 1, hf = pt & 1;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int ch = 4 * hf + q4;
-                    float t8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int col = 8 * ch + e;
-                        t8[e] = (col <= r) ? Tf[r * AFP + col] : 0.f;
-                    }
-                    tc::st_shared_v4(tp + tc::sw128_off(r, ch), tc::pack_bf16(t8[0], t8[1]),
-                                     tc::pack_bf16(t8[2], t8[3]), tc::pack_bf16(t8[4], t8[5]),
-                                     tc::pack_bf16(t8[6], t8[7]));
+            if (pt == 0) {
+                // never leave with a copy or an MMA in flight
+                if (last_loaded >= 0) drain_wait(full, (last_loaded / NPREP) & 1);
+                if (*abort_flag) {
+                    tc::mma_commit(&bars[B_DRAIN]);
+                    drain_wait(&bars[B_DRAIN], 0);
                 }
-            }
-            tc::fence_async_smem();
-            tc::named_bar(1, 128);
-            if (pt == 0) tc::mbar_arrive(&pfull[b]);
-        }
-        if (pt == 0 && *abort_flag) {
-            // drain any MMA still running before tensor memory is released
-            tc::mma_commit(mDrainP);
-            const uint32_t a = smem_u32(mDrainP);
-            for (uint32_t i = 0; i < kPolls && !mbar_try_wait(a, 0); ++i) {
             }
         }
-    } else if (warp >= 8) {
-        // ------------------------------------------------------------ chain
-        const int ct = threadIdx.x - 256, cw = warp - 8;
-        const uint32_t lane_base = (uint32_t)(32 * cw) << 16;
-        const int64_t hrow = ((int64_t)(seq * H + head) * KD + ct) * VD + v0;
-        float h[64];
+    } else {
+        // =============================================================== chain
+        const int ct = threadIdx.x, wg = warp >> 2, q = warp & 3;  // wg: 32 value columns
+        const int row = 32 * q + lane;                               // key row / token row
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int atom = wg >> 1, hcol = wg & 1;  // 64-column atom and its half
+        const int v0 = 32 * wg;
+        const int64_t hrow = ((int64_t)(seq * H + head) * KD + row) * VD + v0;
+        float h[32];
         if (p.h0) {
 #pragma unroll
-            for (int j = 0; j < 64; j += 4) {
+            for (int j = 0; j < 32; j += 4) {
                 const float4 t = *reinterpret_cast<const float4*>(p.h0 + hrow + j);
                 h[j] = t.x; h[j + 1] = t.y; h[j + 2] = t.z; h[j + 3] = t.w;
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) h[j] = 0.f;
+            for (int j = 0; j < 32; ++j) h[j] = 0.f;
         }
-        const uint32_t hb = sbase + OFF_HB, rb = sbase + OFF_RB, ub = sbase + OFF_UB,
-                       wb = sbase + OFF_WB;
-        tc::store_row_bf16(hb, ct, h);
+        const uint32_t hb = sbase + C_OFF_HB, rb = sbase + C_OFF_RB, ub = sbase + C_OFF_UB,
+                       wb = sbase + C_OFF_WB;
+        tc::store_half_row_bf16(hb + atom * 16384, row, hcol, h);
+        uint64_t* mH = &bars[B_MH];
+        uint64_t* mU = &bars[B_MU];
+        uint64_t* mD = &bars[B_MD];
+        uint64_t* mO = &bars[B_MO];
+        const uint32_t idH = tc::idesc_bf16(128, 128, 0, 1);
+        const uint32_t idD = tc::idesc_bf16(128, 128, 1, 1);
+        auto issue_load = [&](int c) {
+            const int s = c & 1;
+            const int y = (int)(cs + (int64_t)C * c);
+            uint64_t* full = &bars[B_FULL + s];
+            uint8_t* kq = base + C_OFF_KQ + s * SZ_KQ;
+            tc::mbar_arrive_expect_tx(full, SZ_KQ);
+            tc::tma_load_2d(kq + 0, &p.tm_k, head * KD + 0, y, full);
+            tc::tma_load_2d(kq + 8192, &p.tm_q, head * KD + 0, y, full);
+            tc::tma_load_2d(kq + 16384, &p.tm_k, head * KD + 64, y, full);
+            tc::tma_load_2d(kq + 24576, &p.tm_q, head * KD + 64, y, full);
+        };
+        auto issue_load_v = [&](int c) {
+            const int y = (int)(cs + (int64_t)C * c);
+            uint64_t* fv = &bars[B_FULLV];
+            uint8_t* vt = base + C_OFF_V;
+            tc::mbar_arrive_expect_tx(fv, SZ_V);
+            tc::tma_load_2d(vt + 0, &p.tm_v, head * VD + 0, y, fv);
+            tc::tma_load_2d(vt + 8192, &p.tm_v, head * VD + 64, y, fv);
+        };
+        int last_loaded = -1;
+        if (ct == 0) {
+            tc::prefetch_tmap(&p.tm_q);
+            tc::prefetch_tmap(&p.tm_k);
+            tc::prefetch_tmap(&p.tm_v);
+            for (int c = 0; c < 2 && c < nch; ++c) {
+                issue_load(c);
+                last_loaded = c;
+            }
+            if (nch > 0) issue_load_v(0);
+        }
+        int last_v = nch > 0 ? 0 : -1;
         tc::fence_async_smem();
-        tc::named_bar(2, 128);
-        const uint32_t idH = tc::idesc_bf16(128, 64, 0, 1);
-        const uint32_t idU = tc::idesc_bf16(128, 64, 0, 1);
-        const uint32_t idD = tc::idesc_bf16(128, 64, 1, 1);
+        tc::named_bar(1, 512);
+        const uint32_t r_free0 = tc::mapa(smem_u32(&bars[B_FREE]), 0);
         for (int c = 0; c < nch; ++c) {
-            const int s = c & 1, b = c & 1;
+            const int s = c & 1, j = c % NPREP, n3 = c / NPREP;
             const int64_t t0 = cs + (int64_t)C * c;
             const int len = (int)((ce - t0) < C ? (ce - t0) : C);
-            const uint32_t kq = sbase + OFF_KQ + s * SZ_KQ;
-            const uint32_t tp = sbase + OFF_TP + b * SZ_TP;
-            const uint32_t colH = COL_H + 64u * (c & 1), colO = COL_O + 64u * (c & 1);
-            const Scal* sc = SC + b;
-            wait(&full[s], (c >> 1) & 1, abort_flag);
-            wait(&pfull[b], (c >> 1) & 1, abort_flag);
+            const uint32_t kq = sbase + C_OFF_KQ + s * SZ_KQ;
+            const uint32_t tp = sbase + C_OFF_TP + j * SZ_TP;
+            const uint32_t colH = C_COL_H + 128u * (c & 1);
+            const ChainScal* sc = reinterpret_cast<const ChainScal*>(base + C_OFF_SC) + j;
+            wait(&bars[B_FULL + s], (c >> 1) & 1, abort_flag);
+            wait(&bars[B_TPF + j], n3 & 1, abort_flag, true);
             if (ct == 0) {
+                tc::fence_async_smem();
                 tc::tc_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16(tmem + colH,
                                  tc::sdesc_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                 tc::sdesc_sw128(hb + kk * 2048, 8192, 1024), idH, kk > 0);
+                                 tc::sdesc_sw128(hb + kk * 2048, 16384, 1024), idH, kk > 0);
                 tc::mma_commit(mH);
             }
             wait(mH, c & 1, abort_flag);
             tc::tc_after_sync();
-            if (ct < 64) {
-                // R = beta (V - gamma * K h) for row r = ct
-                const int r = ct;
-                const float br = sc->beta[r], gr = sc->gam[r];
-                const uint32_t vt = sbase + OFF_V + s * SZ_V;
+            if (q < 2) {
+                // R = beta (V - gamma * K h) for token row `row`, this warpgroup's 32 columns
+                wait(&bars[B_FULLV], c & 1, abort_flag);
+                const float br = sc->beta[row], gr = sc->gam[row];
+                const uint32_t vt = sbase + C_OFF_V + atom * 8192;
+                float x[32];
+                tc::tmem_ld32(tmem + lane_base + colH + v0, x);
+                tc::tmem_wait_ld();
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float x[32];
-                    tc::tmem_ld32(tmem + lane_base + colH + 32 * hf, x);
-                    tc::tmem_wait_ld();
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int ch = 4 * hcol + q4;
+                    const uint4 raw = tc::ld_shared_v4(vt + tc::sw128_off(row, ch));
+                    const __nv_bfloat162* vv = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int ch = 4 * hf + q4;
-                        const uint4 raw = tc::ld_shared_v4(vt + tc::sw128_off(r, ch));
-                        const __nv_bfloat162* vv = reinterpret_cast<const __nv_bfloat162*>(&raw);
-                        float o8[8];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(vv[e]);
-                            o8[2 * e] = br * (f.x - gr * x[8 * q4 + 2 * e]);
-                            o8[2 * e + 1] = br * (f.y - gr * x[8 * q4 + 2 * e + 1]);
-                        }
-                        tc::st_shared_v4(rb + tc::sw128_off(r, ch), tc::pack_bf16(o8[0], o8[1]),
-                                         tc::pack_bf16(o8[2], o8[3]), tc::pack_bf16(o8[4], o8[5]),
-                                         tc::pack_bf16(o8[6], o8[7]));
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(vv[e]);
+                        x[8 * q4 + 2 * e] = br * (f.x - gr * x[8 * q4 + 2 * e]);
+                        x[8 * q4 + 2 * e + 1] = br * (f.y - gr * x[8 * q4 + 2 * e + 1]);
                     }
                 }
+                tc::store_half_row_bf16(rb + atom * 8192, row, hcol, x);
             }
+            if (q == 2 && lane == 0) tc::bulk_wait_read0();  // last chunk's output staging read
             tc::fence_async_smem();
             tc::tc_before_sync();
-            tc::named_bar(2, 128);
+            tc::named_bar(1, 512);
             if (ct == 0) {
                 tc::tc_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + COL_U, tc::sdesc_sw128(tp + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(rb + kk * 2048, 8192, 1024), idU, kk > 0);
+                    tc::mma_bf16(tmem + C_COL_U, tc::sdesc_sw128(tp + kk * 32, 16, 1024),
+                                 tc::sdesc_sw128(rb + kk * 2048, 8192, 1024), idH, kk > 0);
                 tc::mma_commit(mU);
+                if (c + 1 < nch) {  // this chunk's V has been read: fetch the next one
+                    issue_load_v(c + 1);
+                    last_v = c + 1;
+                }
             }
             wait(mU, c & 1, abort_flag);
             tc::tc_after_sync();
-            if (ct < 64) {
-                const int r = ct;
-                const float wr = sc->w[r];
+            if (q < 2) {
+                const float wr = sc->w[row];
+                float x[32];
+                tc::tmem_ld32(tmem + lane_base + C_COL_U + v0, x);
+                tc::tmem_wait_ld();
+                tc::store_half_row_bf16(ub + atom * 8192, row, hcol, x);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float x[32];
-                    tc::tmem_ld32(tmem + lane_base + COL_U + 32 * hf, x);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int ch = 4 * hf + q4;
-                        const float* u = x + 8 * q4;
-                        tc::st_shared_v4(ub + tc::sw128_off(r, ch), tc::pack_bf16(u[0], u[1]),
-                                         tc::pack_bf16(u[2], u[3]), tc::pack_bf16(u[4], u[5]),
-                                         tc::pack_bf16(u[6], u[7]));
-                        tc::st_shared_v4(wb + tc::sw128_off(r, ch),
-                                         tc::pack_bf16(wr * u[0], wr * u[1]),
-                                         tc::pack_bf16(wr * u[2], wr * u[3]),
-                                         tc::pack_bf16(wr * u[4], wr * u[5]),
-                                         tc::pack_bf16(wr * u[6], wr * u[7]));
-                    }
-                }
+                for (int e = 0; e < 32; ++e) x[e] *= wr;
+                tc::store_half_row_bf16(wb + atom * 8192, row, hcol, x);
             }
             tc::fence_async_smem();
             tc::tc_before_sync();
-            tc::named_bar(2, 128);
+            tc::named_bar(1, 512);
             if (ct == 0) {
                 tc::tc_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + COL_D, tc::sdesc_sw128(kq + kk * 2048, 16384, 1024),
+                    tc::mma_bf16(tmem + C_COL_D, tc::sdesc_sw128(kq + kk * 2048, 16384, 1024),
                                  tc::sdesc_sw128(wb + kk * 2048, 8192, 1024), idD, kk > 0);
                 tc::mma_commit(mD);
+            } else if (ct == 64) {
+                // the output product is off the chain: issued by an output-warp thread
+                tc::tc_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + colO, tc::sdesc_sw128(tp + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(ub + kk * 2048, 8192, 1024), idU, kk > 0);
+                    tc::mma_bf16(tmem + C_COL_U, tc::sdesc_sw128(tp + kk * 32, 16, 1024),
+                                 tc::sdesc_sw128(ub + kk * 2048, 8192, 1024), idH, kk > 0);
                 tc::mma_commit(mO);
             }
             wait(mD, c & 1, abort_flag);
@@ -592,97 +652,101 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             {
                 // h <- 2^G2_L h + K^T (w Ut), then the bf16 copy for the next chunk
                 const float e = sc->eGL;
+                float x[32];
+                tc::tmem_ld32(tmem + lane_base + C_COL_D + v0, x);
+                tc::tmem_wait_ld();
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float x[32];
-                    tc::tmem_ld32(tmem + lane_base + COL_D + 32 * hf, x);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) h[32 * hf + j] = fmaf(e, h[32 * hf + j], x[j]);
-                }
-                tc::store_row_bf16(hb, ct, h);
+                for (int jj = 0; jj < 32; ++jj) h[jj] = fmaf(e, h[jj], x[jj]);
+                tc::store_half_row_bf16(hb + atom * 16384, row, hcol, h);
             }
-            if (ct == 0) tc::mbar_arrive(&empty[s]);  // stage no longer read by the chain
+            if (ct == 0 && c + 2 < nch) {
+                // K/Q of this stage are no longer read (MMA_H, MMA_dH done)
+                issue_load(c + 2);
+                last_loaded = c + 2;
+            }
             tc::fence_async_smem();
             tc::tc_before_sync();
-            tc::named_bar(2, 128);
-            if (ct >= 64) {
-                // output rows of this chunk: O = scale (gamma QH + P Ut)
-                const int r = ct - 64;
+            tc::named_bar(1, 512);
+            if (q >= 2) {
+                // output rows: O = scale (gamma QH + P Ut)
+                const int r = row - 64;
                 wait(mO, c & 1, abort_flag);
                 tc::tc_after_sync();
                 const float gr = sc->gam[r], scl = p.scale;
-                float* ost = reinterpret_cast<float*>(base + OFF_OS);
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float qh[32], pu[32];
-                    tc::tmem_ld32(tmem + lane_base + colH + 32 * hf, qh);
-                    tc::tmem_ld32(tmem + lane_base + colO + 32 * hf, pu);
-                    tc::tmem_wait_ld();
-                    float* orow = ost + r * OSP + 32 * hf;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4*>(orow + j) =
-                            make_float4(scl * fmaf(gr, qh[j], pu[j]),
-                                        scl * fmaf(gr, qh[j + 1], pu[j + 1]),
-                                        scl * fmaf(gr, qh[j + 2], pu[j + 2]),
-                                        scl * fmaf(gr, qh[j + 3], pu[j + 3]));
-                }
-                tc::named_bar(3, 64);
-                // coalesced stores: consecutive threads cover consecutive 16-byte
-                // pieces of one output row
-                const int ot = ct - 64;
-                if constexpr (OBF16) {
-                    __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.o);
-#pragma unroll 2
-                    for (int it = 0; it < 8; ++it) {
-                        const int rr = 8 * it + (ot >> 3), c8 = 8 * (ot & 7);
-                        if (rr < len) {
-                            const float4 a = *reinterpret_cast<const float4*>(ost + rr * OSP + c8);
-                            const float4 bq =
-                                *reinterpret_cast<const float4*>(ost + rr * OSP + c8 + 4);
-                            uint4 w4;
-                            w4.x = tc::pack_bf16(a.x, a.y);
-                            w4.y = tc::pack_bf16(a.z, a.w);
-                            w4.z = tc::pack_bf16(bq.x, bq.y);
-                            w4.w = tc::pack_bf16(bq.z, bq.w);
-                            *reinterpret_cast<uint4*>(obase + ((t0 + rr) * H + head) * VD + v0 +
-                                                      c8) = w4;
-                        }
-                    }
-                } else {
-                    float* obase = static_cast<float*>(p.o);
-#pragma unroll 4
-                    for (int it = 0; it < 16; ++it) {
-                        const int rr = 4 * it + (ot >> 4), c4 = 4 * (ot & 15);
-                        if (rr < len)
-                            *reinterpret_cast<float4*>(obase + ((t0 + rr) * H + head) * VD + v0 +
-                                                       c4) =
-                                *reinterpret_cast<const float4*>(ost + rr * OSP + c4);
-                    }
-                }
+                float qh[32], pu[32];
+                tc::tmem_ld32(tmem + lane_base + colH + v0, qh);
+                tc::tmem_ld32(tmem + lane_base + C_COL_U + v0, pu);
+                tc::tmem_wait_ld();
+                // slot j (T, P, gate factors) is consumed once MMA_O is done and
+                // gamma read: hand it back to prep before the stores
                 tc::tc_before_sync();
-                tc::mbar_arrive(&pempty[b]);
+                tc::named_bar(6, 256);
+                if (ct == 64) tc::mbar_arrive_cluster(r_free0 + 8 * j);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) qh[jj] = scl * fmaf(gr, qh[jj], pu[jj]);
+                if (!OBF16 && len == C) {
+                    // full chunk: stage this warpgroup's 64 x 32 fp32 block in the
+                    // 128-byte swizzle layout (the Ut / wUt buffers are free once
+                    // MMA_dH and MMA_O have completed) and let TMA store it
+                    const uint32_t stg = sbase + C_OFF_OS + wg * 8192;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        tc::st_shared_v4(stg + tc::sw128_off(r, ch), __float_as_uint(qh[4 * ch]),
+                                         __float_as_uint(qh[4 * ch + 1]),
+                                         __float_as_uint(qh[4 * ch + 2]),
+                                         __float_as_uint(qh[4 * ch + 3]));
+                    tc::fence_async_smem();
+                    tc::named_bar(2 + wg, 64);
+                    if (q == 2 && lane == 0) {
+                        tc::tma_store_2d(&p.tm_o, stg, head * VD + v0, (int)t0);
+                        tc::bulk_commit();
+                    }
+                } else if (r < len) {
+                    // a sequence's ragged last chunk (or bf16 output): direct row stores
+                    const int64_t orow = ((t0 + r) * H + head) * VD + v0;
+                    if constexpr (OBF16) {
+                        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow;
+#pragma unroll
+                        for (int jj = 0; jj < 32; jj += 8) {
+                            uint4 w4;
+                            w4.x = tc::pack_bf16(qh[jj], qh[jj + 1]);
+                            w4.y = tc::pack_bf16(qh[jj + 2], qh[jj + 3]);
+                            w4.z = tc::pack_bf16(qh[jj + 4], qh[jj + 5]);
+                            w4.w = tc::pack_bf16(qh[jj + 6], qh[jj + 7]);
+                            *reinterpret_cast<uint4*>(op + jj) = w4;
+                        }
+                    } else {
+                        float* op = static_cast<float*>(p.o) + orow;
+#pragma unroll
+                        for (int jj = 0; jj < 32; jj += 4)
+                            *reinterpret_cast<float4*>(op + jj) =
+                                make_float4(qh[jj], qh[jj + 1], qh[jj + 2], qh[jj + 3]);
+                    }
+                }
             }
         }
+        if (q == 2 && lane == 0) tc::bulk_wait0();  // output stores complete
         if (p.hT) {
             float* dst = p.hT + hrow;
 #pragma unroll
-            for (int j = 0; j < 64; j += 4)
-                *reinterpret_cast<float4*>(dst + j) = make_float4(h[j], h[j + 1], h[j + 2], h[j + 3]);
+            for (int jj = 0; jj < 32; jj += 4)
+                *reinterpret_cast<float4*>(dst + jj) = make_float4(h[jj], h[jj + 1], h[jj + 2], h[jj + 3]);
         }
-        if (ct == 0 && *abort_flag) {
-            // drain any MMA still running before tensor memory is released
-            tc::mma_commit(mDrain);
-            const uint32_t a = smem_u32(mDrain);
-            for (uint32_t i = 0; i < kPolls && !mbar_try_wait(a, 0); ++i) {
+        if (ct == 0) {
+            for (int c = (last_loaded > 0 ? last_loaded - 1 : 0); c <= last_loaded && c < nch; ++c)
+                if (c >= 0) drain_wait(&bars[B_FULL + (c & 1)], (c >> 1) & 1);
+            if (last_v >= 0) drain_wait(&bars[B_FULLV], last_v & 1);
+            if (*abort_flag) {
+                tc::mma_commit(&bars[B_DRAIN]);
+                drain_wait(&bars[B_DRAIN], 0);
             }
         }
     }
     tc::tc_before_sync();
     __syncthreads();
+    tc::cluster_sync();  // no CTA leaves while the other may still touch its memory
     tc::tc_after_sync();
-    if (warp == 0) tc::tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 0) tc::tmem_dealloc(tmem, ncols);
 }
 
 using EncodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
@@ -700,30 +764,36 @@ inline EncodeTiled get_encode() {
     return fn;
 }
 
-// [rows, cols] bf16 row-major, box of 64 rows x 64 columns, 128-byte swizzle.
-inline bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+// [rows, cols] row-major, 128-byte swizzle; bf16 inputs use 64 x 64 boxes,
+// the fp32 output 32-column x 64-row boxes.
+inline bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
+                     bool f32 = false) {
     EncodeTiled enc = get_encode();
     if (!enc) return false;
+    const uint64_t esz = f32 ? 4 : 2;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 64};
+    cuuint64_t strides[1] = {cols * esz};
+    cuuint32_t box[2] = {f32 ? 32u : 64u, 64u};
     cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace tcf
 
-// Launches the fused kernel for (n_seq, H) with two value slices.  Returns 0 on
-// success, 1 when the tensor maps could not be built, 2 on a launch error.
+// Launches the fused kernel: one cluster of two CTAs per (sequence, head).
+// Returns 0 on success, 1 when the tensor maps could not be built, 2 on a
+// launch error.
 inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cudaStream_t st) {
     tcf::Params p;
     memset(&p, 0, sizeof(p));
     const uint64_t cols = (uint64_t)a.H * 128;
     if (!tcf::make_map(&p.tm_q, a.q, (uint64_t)T_total, cols) ||
         !tcf::make_map(&p.tm_k, a.k, (uint64_t)T_total, cols) ||
-        !tcf::make_map(&p.tm_v, a.v, (uint64_t)T_total, cols))
+        !tcf::make_map(&p.tm_v, a.v, (uint64_t)T_total, cols) ||
+        (!obf16 && !tcf::make_map(&p.tm_o, a.o, (uint64_t)T_total, cols, true)))
         return 1;
     p.g = a.g;
     p.beta = a.beta;
@@ -740,7 +810,20 @@ inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cuda
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tcf::SMEM_BYTES) != cudaSuccess)
         return 2;
-    kern<<<(unsigned)nb, tcf::kThreads, tcf::SMEM_BYTES, st>>>(p);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)nb, 1, 1);
+    cfg.blockDim = dim3(tcf::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = tcf::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return 2;
     return 0;
 }
 
