@@ -2,34 +2,36 @@
 // (bf16 q/k/v, K = V = 128, fp32 state, fp32 accumulation), sm_100a.
 //
 // The three GDN steps of ZzCompute (PyTorch Helion Hackathon gallery entry 11)
-// -- item 4 "Recompute W/U" (in-chunk cumsum, A, T = (I+A)^-1), item 2 "Chunk
-// Forward H" (state recurrence) and item 3 "Chunk Forward O" (chunk output) --
-// run in one launch, so q/k/v/g/beta are read from HBM once and o/h_T written
-// once.  Per chunk (64 tokens, G2 = log2-scaled in-chunk cumsum of g):
-//   S    = [K; Q] K^T                               (MMA, M=128 N=64 K=128)
-//   A    = strictly-lower beta_r 2^(G2_r-G2_s) (K K^T)_rs,  T = (I + A)^-1
-//   P    = lower-incl 2^(G2_r-G2_s) (Q K^T)_rs
-//   [KH; QH] = [K; Q] h                             (MMA, B = bf16 copy of h)
-//   R    = beta (V - 2^G2 * KH)
-//   Ut   = T R             ( = U - W h of the WY form)  (MMA, A = [T; P])
-//   h'   = 2^G2_L h + K^T (2^(G2_L-G2) * Ut)            (MMA, then fp32 update)
-//   O    = scale (2^G2 * QH + P Ut)                      (MMA, A = [T; P])
-//
+// -- item 4 "Recompute W/U" (in-chunk cumsum, A, T = (I+A)^-1, W, U), item 2
+// "Chunk Forward H" (state recurrence) and item 3 "Chunk Forward O" (chunk
+// output) -- run in one launch, so q/k/v/g/beta are read from HBM once and
+// o/h_T written once.  The state is carried transposed, S = h^T (value rows,
+// key columns, the rule's own orientation).  Per chunk (64 tokens, G2 =
+// log2-scaled in-chunk cumsum of g, w_t = 2^(G2_L - G2_t)):
+//   A   = strictly-lower beta_r 2^(G2_r-G2_s) (K K^T)_rs,  T = (I + A)^-1
+//   P   = lower-incl 2^(G2_r-G2_s) (Q K^T)_rs
+//   Tb  = T diag(beta),  W = T diag(beta 2^G2) K
+//   Ut^T = V^T Tb^T - S W^T                      ( = (U - W h)^T of the WY form)
+//   S'  = 2^G2_L S + (w Ut)^T K
+//   o_t = scale (2^G2_t (S Q^T)_{:,t} + (Ut^T P^T)_{:,t})
 // Each (sequence, head) runs on a cluster of two CTAs, one per SM:
-//  * rank 0, "prep": three warpgroups, each owning every third chunk, its own
-//    TMA stage and its own slot in the chain CTA.  A warpgroup computes S on
-//    tcgen05, the A and P rows, and T by 16x16 blocks, and writes T, P (bf16)
-//    and the per-row gate factors straight into the chain CTA's shared memory
-//    (DSMEM), then releases them with cluster-scope mbarrier arrives.  Three
-//    chunks are in flight, so the serial triangular inverse is off the chain.
-//  * rank 1, "chain": four warpgroups, one per 32 value columns, carry the
-//    fp32 state in registers (one key row per thread) through the serial part
-//    with N = 128 tcgen05 MMAs and write the output rows.
-// TMA loads are issued by the thread that releases a stage, so no producer
-// warp waits.  Every wait is bounded: a wait that gives up sets the CTA's
-// abort flag (all later waits fall through, so every barrier is still
-// reached), records GDN_ERR_TIMEOUT, and the issuing threads drain their
-// copies and MMAs before tensor memory is released.
+//  * rank 0, "prep": three warpgroups, each owning every third chunk and its
+//    own TMA stage: S_kk = [K; Q] K^T and W on tcgen05, the A and P rows and
+//    T by 16x16 blocks.  It assembles [W | Tb | P] (bf16) and the gate factors
+//    in its own stage as the stage's inputs fall free, and ships them to the
+//    chain CTA's shared memory with one bulk copy that completes on the
+//    chain's mbarrier.
+//  * rank 1, "chain": four warpgroups carry S in fp32 registers (value row =
+//    tensor-memory lane, 32 key columns per warpgroup) and keep its bf16 copy
+//    in tensor memory, where it is the A operand of the chain's MMAs, so the
+//    serial part is two tcgen05 products per chunk with no shared-memory
+//    round trip.  The output comes out of tensor memory transposed: each warp
+//    writes 128 contiguous bytes per token.
+// TMA loads are issued by the thread that frees a stage.  Every wait is
+// bounded: a wait that gives up sets the CTA's abort flag (later waits fall
+// through, so every barrier is still reached), records GDN_ERR_TIMEOUT, and
+// the issuing threads drain their copies and MMAs before tensor memory is
+// released.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -46,76 +48,95 @@ namespace tcf {
 constexpr int C = 64;    // chunk
 constexpr int KD = 128;  // key dim
 constexpr int VD = 128;  // value dim
-constexpr int kThreads = 512;
+constexpr int kThreads = 576;  // 16 warps of warpgroup work, an MMA warp and a TMA warp
 constexpr int NPREP = 3;  // prep warpgroups (chunks in flight in the prep CTA)
 constexpr uint32_t kPolls = 1u << 22;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// ---- shared memory, prep CTA (byte offsets from a 1024-aligned base)
-constexpr uint32_t SZ_KQ = 32768;  // [2 key halves][K rows 0-63 | Q rows 64-127][128 B]
+// ---- shared memory, prep CTA
+// The stage holds [K half 0 | Q half 0 | K half 1 | Q half 1] (8 KB each) as
+// loaded; as its parts fall free it is rewritten in place into the slot image
+// sent to the chain CTA: [W half 0 | W half 1 | Tb | P].
+constexpr uint32_t SZ_KQ = 32768;
 constexpr int AFP = 68;            // fp32 row pitch of A / T
 constexpr int XTP = 24;            // pitch of the 16x16 temporaries (conflict-free B fragments)
 constexpr uint32_t SZ_AF = 64 * AFP * 4;
 constexpr uint32_t SZ_XT = 3 * 16 * XTP * 4;
-struct PrepScal {   // per prep warpgroup
-    float G2[64];   // in-chunk inclusive cumsum of g, log2 units
-    float ginv[64]; // 2^-G2 (only when the chunk's decay stays in fp32 range)
-    float gam[64];  // 2^G2
-    float pad;
+struct PrepScal {    // per prep warpgroup
+    float G2[64];    // in-chunk inclusive cumsum of g, log2 units
+    float ginv[64];  // 2^-G2 (only when the chunk's decay stays in fp32 range)
+    float gam[64];   // 2^G2
+    float beta[64];
     float scan_tmp;
-    float pad2[2];
+    float pad[3];
 };
-constexpr uint32_t P_OFF_KQ = 0;                                  // NPREP stages
-constexpr uint32_t P_OFF_AF = P_OFF_KQ + NPREP * SZ_KQ;           // NPREP x A
-constexpr uint32_t P_OFF_TF = P_OFF_AF + NPREP * SZ_AF;           // NPREP x T
-constexpr uint32_t P_OFF_XT = P_OFF_TF + NPREP * SZ_AF;           // NPREP x temporaries
-constexpr uint32_t P_OFF_SC = P_OFF_XT + NPREP * SZ_XT;           // NPREP x PrepScal
-constexpr uint32_t P_END = P_OFF_SC + NPREP * sizeof(PrepScal);
+constexpr uint32_t P_OFF_KQ = 0;                                   // NPREP stages
+constexpr uint32_t P_OFF_AF = P_OFF_KQ + NPREP * SZ_KQ;            // NPREP x A
+constexpr uint32_t P_OFF_TF = P_OFF_AF + NPREP * SZ_AF;            // NPREP x T
+constexpr uint32_t P_OFF_XT = P_OFF_TF + NPREP * SZ_AF;            // NPREP x temporaries
+constexpr uint32_t P_OFF_SC = P_OFF_XT + NPREP * SZ_XT;            // NPREP x PrepScal
+constexpr uint32_t P_OFF_CS = P_OFF_SC + NPREP * sizeof(PrepScal); // NPREP x staged gate factors
+constexpr uint32_t P_END = P_OFF_CS + NPREP * 528;
 
 // ---- shared memory, chain CTA
-constexpr uint32_t SZ_V = 16384;   // [2 atoms of 64 v][64 rows][128 B]
-constexpr uint32_t SZ_TP = 16384;  // [T rows 0-63 | P rows 64-127][64 bf16]
-struct ChainScal {  // per slot, written by the prep CTA
-    float beta[64];
-    float gam[64];  // 2^G2
+// K, V and Q each have two buffers of [2 halves][64 tokens][128 B]: a K buffer
+// is free once dS of its chunk is done, a V buffer once U0 is, a Q buffer once
+// S Q^T is, so each tile is fetched more than a chunk ahead of its use.
+constexpr uint32_t SZ_T = 16384;
+constexpr uint32_t SZ_SLOT = 32768;  // slot: W [2 key halves][64][128 B] | Tb [64][128 B] | P [64][128 B]
+constexpr uint32_t SL_W = 0, SL_TB = 16384, SL_P = 24576;
+constexpr uint32_t SZ_OS = 32768;    // output stage: 4 boxes [64 tokens][32 values fp32], 128B swizzle
+struct ChainScal {  // per slot, written by the prep CTA (bulk copy)
     float w[64];    // 2^(G2_L - G2)
+    float gam[64];  // 2^G2
     float eGL;      // 2^G2_L
     float pad[3];
 };
-constexpr uint32_t C_OFF_KQ = 0;                                // 2 stages
-constexpr uint32_t C_OFF_V = C_OFF_KQ + 2 * SZ_KQ;              // 1 buffer (refilled after R)
-constexpr uint32_t C_OFF_TP = C_OFF_V + SZ_V;                   // NPREP slots
-constexpr uint32_t C_OFF_HB = C_OFF_TP + NPREP * SZ_TP;         // h bf16 [2 atoms][128][128 B]
-constexpr uint32_t C_OFF_RB = C_OFF_HB + 32768;                 // R [2 atoms][64][128 B]
-constexpr uint32_t C_OFF_UB = C_OFF_RB + 16384;                 // Ut
-constexpr uint32_t C_OFF_WB = C_OFF_UB + 16384;                 // 2^(G2_L-G2) Ut
-constexpr uint32_t C_OFF_OS = C_OFF_UB;                         // fp32 output rows [64][128]
-constexpr uint32_t C_OFF_SC = C_OFF_WB + 16384;                 // NPREP x ChainScal
+constexpr uint32_t C_OFF_K = 0;                                 // 2 buffers each
+constexpr uint32_t C_OFF_V = C_OFF_K + 2 * SZ_T;
+constexpr uint32_t C_OFF_Q = C_OFF_V + 2 * SZ_T;
+constexpr uint32_t C_OFF_SL = C_OFF_Q + 2 * SZ_T;               // NPREP slots
+constexpr uint32_t C_OFF_OS = C_OFF_SL + NPREP * SZ_SLOT;
+constexpr uint32_t C_OFF_SC = C_OFF_OS + SZ_OS;                 // NPREP x ChainScal
 constexpr uint32_t C_END = C_OFF_SC + NPREP * sizeof(ChainScal);
 
 constexpr uint32_t BODY = (P_END > C_END ? P_END : C_END);
 constexpr uint32_t OFF_BAR = (BODY + 15) & ~15u;
-constexpr uint32_t OFF_MISC = OFF_BAR + 32 * 8;
+constexpr int NBARS = 40;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(sizeof(ChainScal) == 528, "gate-factor image size");
 
 // ---- tensor memory columns
-constexpr uint32_t P_COL_S = 0;  // NPREP x 64 in the prep CTA
-constexpr uint32_t P_TMEM_COLS = 256;
-constexpr uint32_t C_COL_H = 0;    // two buffers of 128
-constexpr uint32_t C_COL_U = 256;  // Ut, then [T Ut; P Ut]
-constexpr uint32_t C_COL_D = 384;  // K^T (w Ut)
+constexpr uint32_t P_TMEM_COLS = 512;  // prep: per warpgroup 128 (S_kk, then W)
+constexpr uint32_t C_COL_SB = 0;       // chain: bf16 S (128 keys packed in 64 columns)
+constexpr uint32_t C_COL_U = 64;       // Ut^T fp32 (64 tokens)
+constexpr uint32_t C_COL_UB = 128;     // Ut^T bf16 (32)
+constexpr uint32_t C_COL_WB = 160;     // (w Ut)^T bf16 (32)
+constexpr uint32_t C_COL_DS = 192;     // dS fp32 (128 keys)
+constexpr uint32_t C_COL_O1 = 320;     // (S Q^T) fp32, two buffers of 64
+constexpr uint32_t C_COL_O2 = 448;     // (Ut^T P^T) fp32 (64)
 constexpr uint32_t C_TMEM_COLS = 512;
 
 // barrier slots
 enum : int {
-    B_FULL = 0,        // [NPREP] prep: TMA stage; chain uses [0..1]
-    B_MS = 3,          // [NPREP] prep: S ready
-    B_FREE = 6,        // [NPREP] prep: chain slot free (remote arrivals)
-    B_TPF = 9,         // [NPREP] chain: slot filled (remote arrivals, 128 each)
-    B_MH = 12, B_MU, B_MD, B_MO, B_DRAIN,
-    B_FULLV,           // chain: V tile
+    B_FULL = 0,   // [NPREP] prep: TMA stage; chain uses [0..1]
+    B_MS = 3,     // [NPREP] prep: S_kk ready
+    B_FREE = 6,   // [NPREP] prep: chain slot free (remote arrivals)
+    B_TPF = 9,    // [NPREP] chain: slot filled (bulk-copy transactions)
+    B_MW = 12,    // [NPREP] prep: W ready
+    B_MA = 15, B_MD, B_MO, B_DRAIN, B_DRAINP,
+    B_S2,         // chain: Ut^T written (16 warp arrivals)
+    B_S4,         // chain: bf16 S written (16 warp arrivals)
+    B_VF,         // [2] chain: V tile loaded (K tiles use B_FULL 0..1)
+    B_QF = B_VF + 2,  // [2] chain: Q tile loaded
+    B_KFREE = B_QF + 2,     // [2] chain: K buffer read (dS issued before the commit)
+    B_QFREE = B_KFREE + 2,  // [2] chain: Q buffer read (S Q^T)
+    B_VFREE = B_QFREE + 2,  // [2] chain: V buffer read (U0)
+    B_SLOTDONE = B_VFREE + 2,  // [NPREP] chain: slot consumed (MMA commit + 16 warp arrivals)
 };
+static_assert(B_SLOTDONE + NPREP <= NBARS, "barrier slots");
 
 struct Params {
     CUtensorMap tm_q, tm_k, tm_v, tm_o;  // tm_o: fp32 output, 32 x 64 boxes
@@ -152,6 +173,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t phase) {
     for (uint32_t i = 0; i < kPolls && !mbar_try_wait(a, phase); ++i) {
     }
 }
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return tc::pack_bf16(lo, hi); }
 
 // 16x16x16 block product on one warp with the warp-level tf32 tensor-core MMA
 // (m16n8k8, fp32 accumulate): C (+)= X Y for fp32 X, Y in shared memory (row
@@ -298,10 +321,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
     const int nch = (int)((ce - cs + C - 1) / C);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 32; ++i)
-            mbar_init(&bars[i], (i >= B_TPF && i < B_TPF + NPREP) ? 128u : 1u);
+        for (int i = 0; i < NBARS; ++i)
+            mbar_init(&bars[i], (i == B_S2 || i == B_S4)                           ? 16u
+                                : (i >= B_SLOTDONE && i < B_SLOTDONE + NPREP) ? 17u
+                                                                              : 1u);
         misc[1] = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        // chain: arm the slot barriers for the first images before the prep CTA
+        // can start a copy (it waits at the cluster barrier below)
+        if (rank == 1)
+            for (int i = 0; i < NPREP; ++i)
+                tc::mbar_arrive_expect_tx(&bars[B_TPF + i], SZ_SLOT + (uint32_t)sizeof(ChainScal));
     }
     const uint32_t ncols = rank == 0 ? P_TMEM_COLS : C_TMEM_COLS;
     if (warp == 0) tc::tmem_alloc(&misc[0], ncols);
@@ -313,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
 
     if (rank == 0) {
         // ================================================================ prep
-        const int wg = warp >> 2;  // 0..3; warpgroups 1..NPREP work
+        const int wg = warp >> 2;  // warpgroups 1..NPREP work
         if (wg >= 1 && wg <= NPREP) {
             const int pg = wg - 1, pt = threadIdx.x - 128 * wg, pw = warp & 3;
             const int bid = 1 + pg;
@@ -325,12 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             PrepScal* ls = reinterpret_cast<PrepScal*>(base + P_OFF_SC) + pg;
             uint64_t* full = &bars[B_FULL + pg];
             uint64_t* mS = &bars[B_MS + pg];
+            uint64_t* mW = &bars[B_MW + pg];
             uint64_t* sfree = &bars[B_FREE + pg];
-            // the chain CTA's slot for this warpgroup
-            const uint32_t r_tp = tc::mapa(sbase + C_OFF_TP + pg * SZ_TP, 1);
+            const uint32_t tcol = tmem + 128u * pg;  // S_kk (64 columns), then W (128)
+            // this warpgroup's slot in the chain CTA, and the staged gate factors
+            const uint32_t r_sl = tc::mapa(sbase + C_OFF_SL + pg * SZ_SLOT, 1);
             const uint32_t r_sc = tc::mapa(sbase + C_OFF_SC + pg * (uint32_t)sizeof(ChainScal), 1);
             const uint32_t r_tpf = tc::mapa(smem_u32(&bars[B_TPF + pg]), 1);
+            ChainScal* cst = reinterpret_cast<ChainScal*>(base + P_OFF_CS + pg * 528);
+            const uint32_t cst_u32 = sbase + P_OFF_CS + pg * 528;
             const uint32_t idS = tc::idesc_bf16(128, 64, 0, 0);
+            const uint32_t idW = tc::idesc_bf16(128, 128, 0, 1);
             auto issue_load = [&](int c) {
                 const int y = (int)(cs + (int64_t)C * c);
                 tc::mbar_arrive_expect_tx(full, SZ_KQ);
@@ -360,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        tc::mma_bf16(tmem + P_COL_S + 64 * pg, tc::sdesc_sw128(kq + off, 16, 1024),
+                        tc::mma_bf16(tcol, tc::sdesc_sw128(kq + off, 16, 1024),
                                      tc::sdesc_sw128(kq + off, 16, 1024), idS, kk > 0);
                     }
                     tc::mma_commit(mS);
@@ -373,7 +408,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     if (lane >= off) x += y;
                 }
                 if (pt == 31) ls->scan_tmp = x;
-                if (n >= 1) wait(sfree, (n - 1) & 1, abort_flag, true);  // chain done with the slot
                 tc::named_bar(bid, 128);
                 if (pw == 1) x += ls->scan_tmp;
                 if (pt < 64) ls->G2[pt] = x;
@@ -386,27 +420,22 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     const float gm = exp2f(x);
                     ls->gam[pt] = gm;
                     ls->ginv[pt] = factored ? exp2f(-x) : 0.f;
-                    tc::st_cluster_f32(r_sc + 4 * (0 * 64 + pt), bv);
-                    tc::st_cluster_f32(r_sc + 4 * (1 * 64 + pt), gm);
-                    tc::st_cluster_f32(r_sc + 4 * (2 * 64 + pt), exp2f(G2L - x));
-                    if (pt == 0) tc::st_cluster_f32(r_sc + 4 * (3 * 64), exp2f(G2L));
+                    ls->beta[pt] = bv;
+                    cst->w[pt] = exp2f(G2L - x);
+                    cst->gam[pt] = gm;
+                    if (pt == 0) cst->eGL = exp2f(G2L);
                 }
-                // S row of this thread: rows 0-63 = K K^T, rows 64-127 = Q K^T
+                // S_kk row of this thread: rows 0-63 = K K^T, rows 64-127 = Q K^T
                 wait(mS, n & 1, abort_flag);
                 tc::tc_after_sync();
                 float sv[64];
                 {
-                    const uint32_t ta = tmem + ((uint32_t)(32 * pw) << 16) + P_COL_S + 64 * pg;
+                    const uint32_t ta = tcol + ((uint32_t)(32 * pw) << 16);
                     tc::tmem_ld32(ta, *reinterpret_cast<float(*)[32]>(sv));
                     tc::tmem_ld32(ta + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
                     tc::tmem_wait_ld();
                 }
-                // the stage is no longer read: fetch this warpgroup's next chunk into it
-                if (pt == 0 && c + NPREP < nch) {
-                    issue_load(c + NPREP);
-                    last_loaded = c + NPREP;
-                }
-                tc::named_bar(bid, 128);  // ginv / gam visible
+                tc::named_bar(bid, 128);  // ginv / gam / beta visible
                 if (pt < 64) {
                     const int r = pt;
                     const float g2r = ls->G2[r], br = bv;
@@ -452,293 +481,367 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                         for (int j = 0; j < 64; ++j)
                             sv[j] = (j <= r) ? exp2f(g2r - ls->G2[j]) * sv[j] : 0.f;
                     }
-                    // P row -> the chain CTA's slot (rows 64-127 of the stacked operand)
+                    // P row -> the slot image (over the stage's second Q half)
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch)
-                        tc::st_cluster_v4(r_tp + 8192 + tc::sw128_off(r, ch),
-                                          tc::pack_bf16(sv[8 * ch + 0], sv[8 * ch + 1]),
-                                          tc::pack_bf16(sv[8 * ch + 2], sv[8 * ch + 3]),
-                                          tc::pack_bf16(sv[8 * ch + 4], sv[8 * ch + 5]),
-                                          tc::pack_bf16(sv[8 * ch + 6], sv[8 * ch + 7]));
+                        tc::st_shared_v4(kq + SL_P + tc::sw128_off(r, ch),
+                                         pack2(sv[8 * ch + 0], sv[8 * ch + 1]),
+                                         pack2(sv[8 * ch + 2], sv[8 * ch + 3]),
+                                         pack2(sv[8 * ch + 4], sv[8 * ch + 5]),
+                                         pack2(sv[8 * ch + 6], sv[8 * ch + 7]));
                 }
                 tc::tc_before_sync();
-                tc::named_bar(bid, 128);
+                tc::named_bar(bid, 128);  // A rows complete
                 invert_unit_lower(Af, Tf, Xt, pw, lane, bid);
+                uint32_t tb_words[16];  // Tb = T diag(beta), placed once W is done
                 {
-                    // T rows -> bf16 (upper part zero) into the chain CTA's slot
+                    // T rows -> T diag(beta 2^G2) over the stage's first Q half (the A
+                    // operand of W); Tb kept in registers
                     const int r = pt >> 1, hf = pt & 1;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         const int ch = 4 * hf + q4;
-                        float t8[8];
+                        float t8[8], u8[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const int col = 8 * ch + e;
-                            t8[e] = (col <= r) ? Tf[r * AFP + col] : 0.f;
+                            const float tv = (col <= r) ? Tf[r * AFP + col] : 0.f;
+                            t8[e] = tv * ls->beta[col];
+                            u8[e] = t8[e] * ls->gam[col];
                         }
-                        tc::st_cluster_v4(r_tp + tc::sw128_off(r, ch), tc::pack_bf16(t8[0], t8[1]),
-                                          tc::pack_bf16(t8[2], t8[3]), tc::pack_bf16(t8[4], t8[5]),
-                                          tc::pack_bf16(t8[6], t8[7]));
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) tb_words[4 * q4 + e] = pack2(t8[2 * e], t8[2 * e + 1]);
+                        tc::st_shared_v4(kq + 8192 + tc::sw128_off(r, ch), pack2(u8[0], u8[1]),
+                                         pack2(u8[2], u8[3]), pack2(u8[4], u8[5]),
+                                         pack2(u8[6], u8[7]));
                     }
                 }
-                // publish: the chain CTA's MMAs read the slot through the async proxy
-                tc::fence_async_cluster();
-                tc::mbar_arrive_cluster(r_tpf);
+                tc::fence_async_smem();
+                tc::tc_before_sync();
+                tc::named_bar(bid, 128);
+                if (pt == 0) {
+                    // W = [T diag(beta 2^G2); junk] K  (M=128, N=128 keys, K=64 tokens)
+                    tc::tc_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tcol, tc::sdesc_sw128(kq + 8192 + kk * 32, 16, 1024),
+                                     tc::sdesc_sw128(kq + kk * 2048, 16384, 1024), idW, kk > 0);
+                    tc::mma_commit(mW);
+                }
+                wait(mW, n & 1, abort_flag);
+                tc::tc_after_sync();
+                if (pw < 2) {
+                    // W row r (keys 0..127) -> bf16 slot image, over K half 0 / the A tile
+                    const int r = pt;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float xw[32];
+                        tc::tmem_ld32(tcol + ((uint32_t)(32 * pw) << 16) + 32 * q4, xw);
+                        tc::tmem_wait_ld();
+                        const int hf = q4 >> 1;
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int ch = 4 * (q4 & 1) + cc;
+                            tc::st_shared_v4(kq + SL_W + hf * 8192 + tc::sw128_off(r, ch),
+                                             pack2(xw[8 * cc + 0], xw[8 * cc + 1]),
+                                             pack2(xw[8 * cc + 2], xw[8 * cc + 3]),
+                                             pack2(xw[8 * cc + 4], xw[8 * cc + 5]),
+                                             pack2(xw[8 * cc + 6], xw[8 * cc + 7]));
+                        }
+                    }
+                }
+                {
+                    // Tb over K half 1 (W has read it)
+                    const int r = pt >> 1, hf = pt & 1;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        tc::st_shared_v4(kq + SL_TB + tc::sw128_off(r, 4 * hf + q4),
+                                         tb_words[4 * q4], tb_words[4 * q4 + 1],
+                                         tb_words[4 * q4 + 2], tb_words[4 * q4 + 3]);
+                }
+                tc::fence_async_smem();
+                tc::tc_before_sync();
+                tc::named_bar(bid, 128);
+                if (pt == 0) {
+                    // hand the slot image to the chain CTA, then reuse the stage
+                    if (n >= 1) wait(sfree, (n - 1) & 1, abort_flag, true);
+                    tc::bulk_s2cluster(r_sl, kq, SZ_SLOT, r_tpf);
+                    tc::bulk_s2cluster(r_sc, cst_u32, (uint32_t)sizeof(ChainScal), r_tpf);
+                    tc::bulk_commit();
+                    tc::bulk_wait_read0();
+                    if (c + NPREP < nch) {
+                        issue_load(c + NPREP);
+                        last_loaded = c + NPREP;
+                    }
+                }
             }
             if (pt == 0) {
                 // never leave with a copy or an MMA in flight
+                tc::bulk_wait0();
                 if (last_loaded >= 0) drain_wait(full, (last_loaded / NPREP) & 1);
                 if (*abort_flag) {
-                    tc::mma_commit(&bars[B_DRAIN]);
-                    drain_wait(&bars[B_DRAIN], 0);
+                    tc::mma_commit(&bars[B_DRAINP]);
+                    drain_wait(&bars[B_DRAINP], 0);
                 }
             }
         }
     } else {
         // =============================================================== chain
-        const int ct = threadIdx.x, wg = warp >> 2, q = warp & 3;  // wg: 32 value columns
-        const int row = 32 * q + lane;                               // key row / token row
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const int atom = wg >> 1, hcol = wg & 1;  // 64-column atom and its half
-        const int v0 = 32 * wg;
-        const int64_t hrow = ((int64_t)(seq * H + head) * KD + row) * VD + v0;
-        float h[32];
-        if (p.h0) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                const float4 t = *reinterpret_cast<const float4*>(p.h0 + hrow + j);
-                h[j] = t.x; h[j + 1] = t.y; h[j + 2] = t.z; h[j + 3] = t.w;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) h[j] = 0.f;
-        }
-        const uint32_t hb = sbase + C_OFF_HB, rb = sbase + C_OFF_RB, ub = sbase + C_OFF_UB,
-                       wb = sbase + C_OFF_WB;
-        tc::store_half_row_bf16(hb + atom * 16384, row, hcol, h);
-        uint64_t* mH = &bars[B_MH];
-        uint64_t* mU = &bars[B_MU];
+        // warps 0-15: four warpgroups, warpgroup wg owns key columns 32wg.. of S and
+        // tokens 16wg.. of the per-chunk tiles; warp 16: MMA and TMA issue
+        uint64_t* mA = &bars[B_MA];
         uint64_t* mD = &bars[B_MD];
         uint64_t* mO = &bars[B_MO];
-        const uint32_t idH = tc::idesc_bf16(128, 128, 0, 1);
-        const uint32_t idD = tc::idesc_bf16(128, 128, 1, 1);
-        auto issue_load = [&](int c) {
-            const int s = c & 1;
-            const int y = (int)(cs + (int64_t)C * c);
-            uint64_t* full = &bars[B_FULL + s];
-            uint8_t* kq = base + C_OFF_KQ + s * SZ_KQ;
-            tc::mbar_arrive_expect_tx(full, SZ_KQ);
-            tc::tma_load_2d(kq + 0, &p.tm_k, head * KD + 0, y, full);
-            tc::tma_load_2d(kq + 8192, &p.tm_q, head * KD + 0, y, full);
-            tc::tma_load_2d(kq + 16384, &p.tm_k, head * KD + 64, y, full);
-            tc::tma_load_2d(kq + 24576, &p.tm_q, head * KD + 64, y, full);
-        };
-        auto issue_load_v = [&](int c) {
-            const int y = (int)(cs + (int64_t)C * c);
-            uint64_t* fv = &bars[B_FULLV];
-            uint8_t* vt = base + C_OFF_V;
-            tc::mbar_arrive_expect_tx(fv, SZ_V);
-            tc::tma_load_2d(vt + 0, &p.tm_v, head * VD + 0, y, fv);
-            tc::tma_load_2d(vt + 8192, &p.tm_v, head * VD + 64, y, fv);
-        };
-        int last_loaded = -1;
-        if (ct == 0) {
-            tc::prefetch_tmap(&p.tm_q);
-            tc::prefetch_tmap(&p.tm_k);
-            tc::prefetch_tmap(&p.tm_v);
-            for (int c = 0; c < 2 && c < nch; ++c) {
-                issue_load(c);
-                last_loaded = c;
-            }
-            if (nch > 0) issue_load_v(0);
-        }
-        int last_v = nch > 0 ? 0 : -1;
-        tc::fence_async_smem();
-        tc::named_bar(1, 512);
-        const uint32_t r_free0 = tc::mapa(smem_u32(&bars[B_FREE]), 0);
-        for (int c = 0; c < nch; ++c) {
-            const int s = c & 1, j = c % NPREP, n3 = c / NPREP;
-            const int64_t t0 = cs + (int64_t)C * c;
-            const int len = (int)((ce - t0) < C ? (ce - t0) : C);
-            const uint32_t kq = sbase + C_OFF_KQ + s * SZ_KQ;
-            const uint32_t tp = sbase + C_OFF_TP + j * SZ_TP;
-            const uint32_t colH = C_COL_H + 128u * (c & 1);
-            const ChainScal* sc = reinterpret_cast<const ChainScal*>(base + C_OFF_SC) + j;
-            wait(&bars[B_FULL + s], (c >> 1) & 1, abort_flag);
-            wait(&bars[B_TPF + j], n3 & 1, abort_flag, true);
-            if (ct == 0) {
-                tc::fence_async_smem();
-                tc::tc_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(tmem + colH,
-                                 tc::sdesc_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                 tc::sdesc_sw128(hb + kk * 2048, 16384, 1024), idH, kk > 0);
-                tc::mma_commit(mH);
-            }
-            wait(mH, c & 1, abort_flag);
-            tc::tc_after_sync();
-            if (q < 2) {
-                // R = beta (V - gamma * K h) for token row `row`, this warpgroup's 32 columns
-                wait(&bars[B_FULLV], c & 1, abort_flag);
-                const float br = sc->beta[row], gr = sc->gam[row];
-                const uint32_t vt = sbase + C_OFF_V + atom * 8192;
-                float x[32];
-                tc::tmem_ld32(tmem + lane_base + colH + v0, x);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int ch = 4 * hcol + q4;
-                    const uint4 raw = tc::ld_shared_v4(vt + tc::sw128_off(row, ch));
-                    const __nv_bfloat162* vv = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(vv[e]);
-                        x[8 * q4 + 2 * e] = br * (f.x - gr * x[8 * q4 + 2 * e]);
-                        x[8 * q4 + 2 * e + 1] = br * (f.y - gr * x[8 * q4 + 2 * e + 1]);
-                    }
+        uint64_t* s2 = &bars[B_S2];
+        uint64_t* s4 = &bars[B_S4];
+        constexpr uint32_t kSlotTx = SZ_SLOT + (uint32_t)sizeof(ChainScal);
+        if (warp == 17) {
+            if (lane == 0) {
+                // TMA warp: K, V and Q tiles (two buffers each, buffer c & 1) as their
+                // buffers fall free, and the slots back to the prep CTA once consumed
+                const uint32_t r_free0 = tc::mapa(smem_u32(&bars[B_FREE]), 0);
+                int last[3] = {-1, -1, -1};
+                auto load = [&](int kind, int c) {
+                    if (*abort_flag) return;  // at most one copy in flight per buffer
+                    const int y = (int)(cs + (int64_t)C * c);
+                    const uint32_t off = (kind == 0 ? C_OFF_K : kind == 1 ? C_OFF_V : C_OFF_Q) +
+                                         (c & 1) * SZ_T;
+                    uint64_t* bar = &bars[(kind == 0 ? B_FULL : kind == 1 ? B_VF : B_QF) + (c & 1)];
+                    const CUtensorMap* m = kind == 0 ? &p.tm_k : kind == 1 ? &p.tm_v : &p.tm_q;
+                    const int x0 = head * (kind == 1 ? VD : KD);
+                    tc::mbar_arrive_expect_tx(bar, SZ_T);
+                    tc::tma_load_2d(base + off, m, x0, y, bar);
+                    tc::tma_load_2d(base + off + 8192, m, x0 + 64, y, bar);
+                    last[kind] = c;
+                };
+                tc::prefetch_tmap(&p.tm_k);
+                tc::prefetch_tmap(&p.tm_v);
+                tc::prefetch_tmap(&p.tm_q);
+                for (int c = 0; c < 2 && c < nch; ++c) {
+                    load(1, c);
+                    load(0, c);
+                    load(2, c);
                 }
-                tc::store_half_row_bf16(rb + atom * 8192, row, hcol, x);
-            }
-            if (q == 2 && lane == 0) tc::bulk_wait_read0();  // last chunk's output staging read
-            tc::fence_async_smem();
-            tc::tc_before_sync();
-            tc::named_bar(1, 512);
-            if (ct == 0) {
-                tc::tc_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + C_COL_U, tc::sdesc_sw128(tp + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(rb + kk * 2048, 8192, 1024), idH, kk > 0);
-                tc::mma_commit(mU);
-                if (c + 1 < nch) {  // this chunk's V has been read: fetch the next one
-                    issue_load_v(c + 1);
-                    last_v = c + 1;
-                }
-            }
-            wait(mU, c & 1, abort_flag);
-            tc::tc_after_sync();
-            if (q < 2) {
-                const float wr = sc->w[row];
-                float x[32];
-                tc::tmem_ld32(tmem + lane_base + C_COL_U + v0, x);
-                tc::tmem_wait_ld();
-                tc::store_half_row_bf16(ub + atom * 8192, row, hcol, x);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] *= wr;
-                tc::store_half_row_bf16(wb + atom * 8192, row, hcol, x);
-            }
-            tc::fence_async_smem();
-            tc::tc_before_sync();
-            tc::named_bar(1, 512);
-            if (ct == 0) {
-                tc::tc_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + C_COL_D, tc::sdesc_sw128(kq + kk * 2048, 16384, 1024),
-                                 tc::sdesc_sw128(wb + kk * 2048, 8192, 1024), idD, kk > 0);
-                tc::mma_commit(mD);
-            } else if (ct == 64) {
-                // the output product is off the chain: issued by an output-warp thread
-                tc::tc_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + C_COL_U, tc::sdesc_sw128(tp + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(ub + kk * 2048, 8192, 1024), idH, kk > 0);
-                tc::mma_commit(mO);
-            }
-            wait(mD, c & 1, abort_flag);
-            tc::tc_after_sync();
-            {
-                // h <- 2^G2_L h + K^T (w Ut), then the bf16 copy for the next chunk
-                const float e = sc->eGL;
-                float x[32];
-                tc::tmem_ld32(tmem + lane_base + C_COL_D + v0, x);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) h[jj] = fmaf(e, h[jj], x[jj]);
-                tc::store_half_row_bf16(hb + atom * 16384, row, hcol, h);
-            }
-            if (ct == 0 && c + 2 < nch) {
-                // K/Q of this stage are no longer read (MMA_H, MMA_dH done)
-                issue_load(c + 2);
-                last_loaded = c + 2;
-            }
-            tc::fence_async_smem();
-            tc::tc_before_sync();
-            tc::named_bar(1, 512);
-            if (q >= 2) {
-                // output rows: O = scale (gamma QH + P Ut)
-                const int r = row - 64;
-                wait(mO, c & 1, abort_flag);
-                tc::tc_after_sync();
-                const float gr = sc->gam[r], scl = p.scale;
-                float qh[32], pu[32];
-                tc::tmem_ld32(tmem + lane_base + colH + v0, qh);
-                tc::tmem_ld32(tmem + lane_base + C_COL_U + v0, pu);
-                tc::tmem_wait_ld();
-                // slot j (T, P, gate factors) is consumed once MMA_O is done and
-                // gamma read: hand it back to prep before the stores
-                tc::tc_before_sync();
-                tc::named_bar(6, 256);
-                if (ct == 64) tc::mbar_arrive_cluster(r_free0 + 8 * j);
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) qh[jj] = scl * fmaf(gr, qh[jj], pu[jj]);
-                if (!OBF16 && len == C) {
-                    // full chunk: stage this warpgroup's 64 x 32 fp32 block in the
-                    // 128-byte swizzle layout (the Ut / wUt buffers are free once
-                    // MMA_dH and MMA_O have completed) and let TMA store it
-                    const uint32_t stg = sbase + C_OFF_OS + wg * 8192;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        tc::st_shared_v4(stg + tc::sw128_off(r, ch), __float_as_uint(qh[4 * ch]),
-                                         __float_as_uint(qh[4 * ch + 1]),
-                                         __float_as_uint(qh[4 * ch + 2]),
-                                         __float_as_uint(qh[4 * ch + 3]));
-                    tc::fence_async_smem();
-                    tc::named_bar(2 + wg, 64);
-                    if (q == 2 && lane == 0) {
-                        tc::tma_store_2d(&p.tm_o, stg, head * VD + v0, (int)t0);
-                        tc::bulk_commit();
+                for (int c = 0; c < nch; ++c) {
+                    const uint32_t ph = (c >> 1) & 1;
+                    if (c + 2 < nch) {
+                        if (wait(&bars[B_VFREE + (c & 1)], ph, abort_flag)) load(1, c + 2);
+                        if (wait(&bars[B_QFREE + (c & 1)], ph, abort_flag)) load(2, c + 2);
+                        if (wait(&bars[B_KFREE + (c & 1)], ph, abort_flag)) load(0, c + 2);
                     }
-                } else if (r < len) {
-                    // a sequence's ragged last chunk (or bf16 output): direct row stores
-                    const int64_t orow = ((t0 + r) * H + head) * VD + v0;
-                    if constexpr (OBF16) {
-                        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow;
-#pragma unroll
-                        for (int jj = 0; jj < 32; jj += 8) {
-                            uint4 w4;
-                            w4.x = tc::pack_bf16(qh[jj], qh[jj + 1]);
-                            w4.y = tc::pack_bf16(qh[jj + 2], qh[jj + 3]);
-                            w4.z = tc::pack_bf16(qh[jj + 4], qh[jj + 5]);
-                            w4.w = tc::pack_bf16(qh[jj + 6], qh[jj + 7]);
-                            *reinterpret_cast<uint4*>(op + jj) = w4;
+                    if (c + NPREP < nch) {
+                        // re-arm the slot's barrier for the next image, then hand the
+                        // slot back to the prep CTA
+                        const int j = c % NPREP;
+                        if (wait(&bars[B_SLOTDONE + j], (c / NPREP) & 1, abort_flag)) {
+                            tc::mbar_arrive_expect_tx(&bars[B_TPF + j], kSlotTx);
+                            tc::mbar_arrive_cluster(r_free0 + 8 * j);
                         }
-                    } else {
-                        float* op = static_cast<float*>(p.o) + orow;
-#pragma unroll
-                        for (int jj = 0; jj < 32; jj += 4)
-                            *reinterpret_cast<float4*>(op + jj) =
-                                make_float4(qh[jj], qh[jj + 1], qh[jj + 2], qh[jj + 3]);
                     }
                 }
+                // never leave with a copy in flight
+                for (int kind = 0; kind < 3; ++kind) {
+                    uint64_t* b0 = &bars[kind == 0 ? B_FULL : kind == 1 ? B_VF : B_QF];
+                    for (int c = last[kind] - 1; c <= last[kind]; ++c)
+                        if (c >= 0) drain_wait(b0 + (c & 1), (c >> 1) & 1);
+                }
             }
-        }
-        if (q == 2 && lane == 0) tc::bulk_wait0();  // output stores complete
-        if (p.hT) {
-            float* dst = p.hT + hrow;
+        } else if (warp == 16) {
+            if (lane == 0) {
+                // MMA warp: the dependent products (U, dS) are issued as soon as their
+                // inputs are written; the output products fill the gaps
+                const uint32_t idU0 = tc::idesc_bf16(128, 64, 1, 0);
+                const uint32_t id1 = tc::idesc_bf16(128, 64, 0, 0) | tc::kNegateA;
+                const uint32_t idO = tc::idesc_bf16(128, 64, 0, 0);
+                const uint32_t id2 = tc::idesc_bf16(128, 128, 0, 1);
+                // U0 for chunk c: D_U = V^T Tb^T  (A = V tile MN-major, B = Tb K-major)
+                auto issue_u0 = [&](int c) {
+                    wait(&bars[B_VF + (c & 1)], (c >> 1) & 1, abort_flag);
+                    wait(&bars[B_TPF + c % NPREP], (c / NPREP) & 1, abort_flag);
+                    tc::tc_after_sync();
+                    const uint32_t vt = sbase + C_OFF_V + (c & 1) * SZ_T;
+                    const uint32_t tb = sbase + C_OFF_SL + (c % NPREP) * SZ_SLOT + SL_TB;
 #pragma unroll
-            for (int jj = 0; jj < 32; jj += 4)
-                *reinterpret_cast<float4*>(dst + jj) = make_float4(h[jj], h[jj + 1], h[jj + 2], h[jj + 3]);
-        }
-        if (ct == 0) {
-            for (int c = (last_loaded > 0 ? last_loaded - 1 : 0); c <= last_loaded && c < nch; ++c)
-                if (c >= 0) drain_wait(&bars[B_FULL + (c & 1)], (c >> 1) & 1);
-            if (last_v >= 0) drain_wait(&bars[B_FULLV], last_v & 1);
-            if (*abort_flag) {
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tmem + C_COL_U, tc::sdesc_sw128(vt + kk * 2048, 8192, 1024),
+                                     tc::sdesc_sw128(tb + kk * 32, 16, 1024), idU0, kk > 0);
+                    tc::mma_commit(&bars[B_VFREE + (c & 1)]);
+                };
+                if (nch > 0) issue_u0(0);
+                for (int c = 0; c < nch; ++c) {
+                    const uint32_t sl = sbase + C_OFF_SL + (c % NPREP) * SZ_SLOT;
+                    wait(s4, c & 1, abort_flag);  // bf16 S of this chunk written
+                    tc::tc_after_sync();
+                    // Ut^T = V^T Tb^T - S W^T
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_bf16_ts(tmem + C_COL_U, tmem + C_COL_SB + 8 * kk,
+                                        tc::sdesc_sw128(sl + SL_W + (kk >> 2) * 8192 + (kk & 3) * 32,
+                                                        16, 1024),
+                                        id1, 1);
+                    tc::mma_commit(mA);
+                    // S Q^T for the output
+                    wait(&bars[B_QF + (c & 1)], (c >> 1) & 1, abort_flag);
+                    tc::tc_after_sync();
+                    const uint32_t qt = sbase + C_OFF_Q + (c & 1) * SZ_T;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_bf16_ts(tmem + C_COL_O1 + 64u * (c & 1), tmem + C_COL_SB + 8 * kk,
+                                        tc::sdesc_sw128(qt + (kk >> 2) * 8192 + (kk & 3) * 32, 16,
+                                                        1024),
+                                        idO, kk > 0);
+                    tc::mma_commit(&bars[B_QFREE + (c & 1)]);
+                    wait(s2, c & 1, abort_flag);  // Ut^T, (w Ut)^T written; output(c-1) done
+                    wait(&bars[B_FULL + (c & 1)], (c >> 1) & 1, abort_flag);
+                    tc::tc_after_sync();
+                    // dS = (w Ut)^T K
+                    const uint32_t kt = sbase + C_OFF_K + (c & 1) * SZ_T;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16_ts(tmem + C_COL_DS, tmem + C_COL_WB + 8 * kk,
+                                        tc::sdesc_sw128(kt + kk * 2048, 8192, 1024), id2, kk > 0);
+                    tc::mma_commit(mD);
+                    tc::mma_commit(&bars[B_KFREE + (c & 1)]);
+                    // Ut^T P^T
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16_ts(tmem + C_COL_O2, tmem + C_COL_UB + 8 * kk,
+                                        tc::sdesc_sw128(sl + SL_P + kk * 32, 16, 1024), idO,
+                                        kk > 0);
+                    tc::mma_commit(mO);
+                    tc::mma_commit(&bars[B_SLOTDONE + c % NPREP]);
+                    // next chunk's U0 (D_U was read before s2)
+                    if (c + 1 < nch) issue_u0(c + 1);
+                }
+                // never leave with an MMA in flight
                 tc::mma_commit(&bars[B_DRAIN]);
                 drain_wait(&bars[B_DRAIN], 0);
+            }
+        } else {
+            const int wg = warp >> 2, q = warp & 3;
+            const int vr = 32 * q + lane;  // value row of S = tensor-memory lane
+            const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+            const int k0 = 32 * wg;        // this warpgroup's 32 key columns of S
+            const int64_t hb0 = (int64_t)(seq * H + head) * KD * VD;
+            // S[vr][k0 .. k0+31] = h[k][vr]
+            float S[32];
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+                S[jj] = p.h0 ? p.h0[hb0 + (int64_t)(k0 + jj) * VD + vr] : 0.f;
+            auto store_sb = [&]() {
+                uint32_t w16[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) w16[jj] = pack2(S[2 * jj], S[2 * jj + 1]);
+                tc::tmem_st16(tmem + lane_base + C_COL_SB + 16u * wg, w16);
+                tc::tmem_wait_st();
+                tc::tc_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(s4);
+            };
+            store_sb();
+            const bool issuer = (wg == 0 && lane == 0);  // one thread per value quarter
+            auto output = [&](int c) {
+                // o_t = scale (2^G2_t (S Q^T)[vr][t] + (Ut^T P^T)[vr][t]) for 16 tokens
+                const int64_t t0 = cs + (int64_t)C * c;
+                const int len = (int)((ce - t0) < C ? (ce - t0) : C);
+                const ChainScal* scp =
+                    reinterpret_cast<const ChainScal*>(base + C_OFF_SC) + (c % NPREP);
+                wait(mO, c & 1, abort_flag);
+                tc::tc_after_sync();
+                float o1[16], o2[16];
+                tc::tmem_ld16(tmem + lane_base + C_COL_O1 + 64u * (c & 1) + 16u * wg, o1);
+                tc::tmem_ld16(tmem + lane_base + C_COL_O2 + 16u * wg, o2);
+                tc::tmem_wait_ld();
+                const float scl = p.scale;
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) o1[jj] = scl * fmaf(scp->gam[16 * wg + jj], o1[jj], o2[jj]);
+                if (!OBF16 && len == C) {
+                    // stage the 64 x 32 block of this value quarter (128-byte swizzle),
+                    // then one TMA store per quarter
+                    const uint32_t stg = sbase + C_OFF_OS + q * 8192;
+                    if (issuer) tc::bulk_wait_read0();  // previous chunk's store read the stage
+                    tc::named_bar(1 + q, 128);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int t = 16 * wg + jj;
+                        asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + tc::sw128_off(t, lane >> 2) +
+                                                                    4 * (lane & 3)),
+                                     "f"(o1[jj])
+                                     : "memory");
+                    }
+                    tc::fence_async_smem();
+                    tc::named_bar(1 + q, 128);
+                    if (issuer) {
+                        tc::tma_store_2d(&p.tm_o, stg, head * VD + 32 * q, (int)t0);
+                        tc::bulk_commit();
+                    }
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int t = 16 * wg + jj;
+                        if (t < len) {
+                            const int64_t oi = ((t0 + t) * H + head) * VD + vr;
+                            if constexpr (OBF16)
+                                static_cast<__nv_bfloat16*>(p.o)[oi] = __float2bfloat16_rn(o1[jj]);
+                            else
+                                static_cast<float*>(p.o)[oi] = o1[jj];
+                        }
+                    }
+                }
+            };
+            // this warp is done with the gate factors of chunk c
+            auto slot_consumed = [&](int c) {
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bars[B_SLOTDONE + c % NPREP]);
+            };
+            for (int c = 0; c < nch; ++c) {
+                const int j = c % NPREP;
+                const ChainScal* sc = reinterpret_cast<const ChainScal*>(base + C_OFF_SC) + j;
+                wait(&bars[B_TPF + j], (c / NPREP) & 1, abort_flag);
+                if (c >= 1) output(c - 1);  // overlaps this chunk's MMA latency
+                if (c >= 1) slot_consumed(c - 1);
+                wait(mA, c & 1, abort_flag);
+                tc::tc_after_sync();
+                {
+                    // Ut^T columns 16wg..16wg+15 -> bf16 Ut^T and (w Ut)^T in tensor memory
+                    float u[16];
+                    tc::tmem_ld16(tmem + lane_base + C_COL_U + 16u * wg, u);
+                    tc::tmem_wait_ld();
+                    uint32_t ub[8], wb[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const float w0 = sc->w[16 * wg + 2 * jj], w1 = sc->w[16 * wg + 2 * jj + 1];
+                        ub[jj] = pack2(u[2 * jj], u[2 * jj + 1]);
+                        wb[jj] = pack2(w0 * u[2 * jj], w1 * u[2 * jj + 1]);
+                    }
+                    tc::tmem_st8(tmem + lane_base + C_COL_UB + 8u * wg, ub);
+                    tc::tmem_st8(tmem + lane_base + C_COL_WB + 8u * wg, wb);
+                    tc::tmem_wait_st();
+                    tc::tc_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(s2);
+                }
+                wait(mD, c & 1, abort_flag);
+                tc::tc_after_sync();
+                {
+                    // S <- 2^G2_L S + dS, and its bf16 copy for the next chunk
+                    const float e = sc->eGL;
+                    float d[32];
+                    tc::tmem_ld32(tmem + lane_base + C_COL_DS + 32u * wg, d);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) S[jj] = fmaf(e, S[jj], d[jj]);
+                    store_sb();  // S Q^T and MMA_1 of this chunk completed before dS
+                }
+            }
+            if (nch >= 1) {
+                output(nch - 1);
+                slot_consumed(nch - 1);
+            }
+            if (issuer) tc::bulk_wait0();  // output stores complete
+            if (p.hT) {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) p.hT[hb0 + (int64_t)(k0 + jj) * VD + vr] = S[jj];
             }
         }
     }
