@@ -15,6 +15,9 @@ Functions and their parity status (pins live in ``tests/test_oracle_pins.py``):
   index order inside each part is a reading (parity unpinned there).
 * ``gdp_decode_step`` -- prepare, then the rule over the M Householder copies.
   Recurrence pinned through ``gdn_fwd``; layout as ``gdp_decode_prepare``.
+* ``conv1d_fwd`` / ``conv1d_update`` -- ZzCompute item 1, causal depthwise conv1d
+  (W = 4) and its one-token update with -1 padding slots (Megatron-Core
+  ``gdp_decode_prepare`` module description).  Pinned.
 """
 from __future__ import annotations
 
@@ -57,6 +60,8 @@ def _load():
         lib.oracle_gdp_decode_step.argtypes = [P, i64, P, i64, P, P, i32, i32, i32, i32, i32, i32,
                                                P, f64, i32, P, P, i32]
         lib.oracle_gdp_decode_step.restype = i32
+        lib.oracle_conv1d_fwd.argtypes = [P, P, P, i32, P, i32, i32, P, i32, P, P]
+        lib.oracle_conv1d_update.argtypes = [P, P, P, i32, P, P, i32, i32, i32, P]
         _lib = lib
     return _lib
 
@@ -188,3 +193,53 @@ def gdp_decode_step(x, ba, A_log, dt_bias, state, M, H, G, P, N, scale=1.0, qk_l
                                                   int(bool(qk_l2norm)), ptr(st_out), ptr(o),
                                                   int(n_threads))
     return o, st_out
+
+
+def conv1d_fwd(x, w, bias=None, cu_seqlens=None, init_state=None, activation=False):
+    """Causal depthwise conv1d in fp64.
+
+    x: [B, T, C] (dense) or [1, T_total, C] with cu_seqlens; w: [C, W]; bias: [C];
+    init_state: [n_seq, C, W-1].  Returns (y fp64 shaped like x, final_state float32
+    [n_seq, C, W-1])."""
+    xs = _f32(x)
+    B, T, C = xs.shape
+    if cu_seqlens is None:
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        assert B == 1
+        cu = cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else np.asarray(cu_seqlens)
+        cu = cu.astype(np.int64)
+    n_seq = len(cu) - 1
+    xs, px = _c(xs, np.float32)
+    w, pw = _c(_f32(w), np.float32)
+    W = w.shape[1]
+    pb = _c(_f32(bias), np.float32) if bias is not None else (None, None)
+    pi = _c(_f32(init_state), np.float32) if init_state is not None else (None, None)
+    cu, pcu = _c(cu, np.int64)
+    y = np.empty((B, T, C), np.float64)
+    fin = np.zeros((n_seq, C, max(W - 1, 1)), np.float32)
+    _load().oracle_conv1d_fwd(px, pw, pb[1], W, pcu, n_seq, C, pi[1], int(bool(activation)),
+                              y.ctypes.data_as(ctypes.c_void_p), fin.ctypes.data_as(ctypes.c_void_p))
+    return y, fin[:, :, :W - 1]
+
+
+def conv1d_update(x, w, state, bias=None, state_idx=None, activation=False):
+    """One-token update: x [n, C]; state [n_slots, C, W-1] (not modified; a new
+    array is returned); state_idx [n] int or None.  Returns (y fp64 [n, C],
+    new_state float32)."""
+    xs, px = _c(_f32(x), np.float32)
+    n, C = xs.shape
+    w, pw = _c(_f32(w), np.float32)
+    W = w.shape[1]
+    st = np.array(_f32(state), dtype=np.float32, copy=True)
+    pst = st.ctypes.data_as(ctypes.c_void_p)
+    pb = _c(_f32(bias), np.float32) if bias is not None else (None, None)
+    if state_idx is not None:
+        idx = state_idx.cpu().numpy() if hasattr(state_idx, "cpu") else np.asarray(state_idx)
+        pidx = _c(idx, np.int32)
+    else:
+        pidx = (None, None)
+    y = np.empty((n, C), np.float64)
+    _load().oracle_conv1d_update(px, pw, pb[1], W, pst, pidx[1], n, C, int(bool(activation)),
+                                 y.ctypes.data_as(ctypes.c_void_p))
+    return y, st

@@ -26,6 +26,18 @@
  *    chunked form of this same map (64-token chunks); the oracle does not
  *    chunk at all, it walks every token in order.
  *
+ *  - Short convolution.  ZzCompute item 1 ("Causal Conv1d -- Depthwise
+ *    Causal Convolution"): every channel is convolved on its own with its
+ *    past context, filter width W = 4, boundaries by masked loads rather
+ *    than padding.  Written out per sequence and channel:
+ *        y[t,c] = bias[c] + sum_{i<W} w[c,i] x[t-(W-1)+i, c],
+ *    so w[c,W-1] weighs the current input; taps before the sequence start
+ *    read the sequence's initial conv state (its W-1 previous inputs, oldest
+ *    first) or zero.  SiLU (y * sigmoid(y)) is an option.  The one-token
+ *    decode update shifts the same W-1 input window; a request whose state
+ *    slot is -1 is padding: its output is zero and no state is touched
+ *    (Megatron-Core "gdp_decode_prepare": "a -1 slot zeroes its conv output").
+ *
  *  - GDP decode.  Megatron-Core "gdp_decode_prepare" (function entry and
  *    parameter list): the post-conv row x = [value | key | query] with sizes
  *    M*H*P, M*G*N, G*N; ba = [b (M*H) | a (H)]; key/query GQA-expanded from
@@ -45,6 +57,11 @@
  *    oracle_gdp_decode_step             : recurrence pinned through
  *                                         oracle_gdn_fwd (same token step);
  *                                         layout as decode_prepare.
+ *    oracle_conv1d_fwd / _update        : pinned (impulse response, numpy's
+ *                                         convolve, constant input, token-
+ *                                         by-token update = whole sequence);
+ *                                         the tap order w[c,W-1] = current
+ *                                         input is a reading.
  */
 #include <math.h>
 #include <pthread.h>
@@ -293,4 +310,61 @@ int oracle_gdp_decode_step(const uint16_t* x, int64_t x_n_stride, const uint16_t
     for (int i = 0; i < nth; ++i) pthread_join(th[i], NULL);
     free(th); free(jobs); free(q); free(k); free(v); free(beta); free(g);
     return nth;
+}
+
+/* ------------------------------------------------------------- short conv */
+
+static double silu_f64(double y) { return y / (1.0 + exp(-y)); }
+
+/* Causal depthwise conv1d over packed sequences (ZzCompute item 1).
+ * x [rows, C] (fp32 values; bf16 inputs widened exactly), rows = cu[n_seq];
+ * w [C, W]; bias [C] or NULL; init [n_seq, C, W-1] or NULL (zeros);
+ * y [rows, C] fp64; final [n_seq, C, W-1] or NULL: the last W-1 inputs of each
+ * sequence, oldest first (initial-state values where the sequence is shorter). */
+void oracle_conv1d_fwd(const float* x, const float* w, const float* bias, int W,
+                       const int64_t* cu, int n_seq, int C, const float* init, int act,
+                       double* y, float* final_state) {
+    const int H = W - 1;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t t0 = cu[s], len = cu[s + 1] - cu[s];
+        for (int c = 0; c < C; ++c) {
+            /* input at sequence position tau (may be negative) */
+#define XIN(tau) ((tau) >= 0 ? (double)x[(t0 + (tau)) * C + c] \
+                             : (init ? (double)init[((int64_t)s * C + c) * H + (H + (tau))] : 0.0))
+            for (int64_t t = 0; t < len; ++t) {
+                double acc = bias ? (double)bias[c] : 0.0;
+                for (int i = 0; i < W; ++i) acc += (double)w[(int64_t)c * W + i] * XIN(t - H + i);
+                y[(t0 + t) * C + c] = act ? silu_f64(acc) : acc;
+            }
+            if (final_state)
+                for (int j = 0; j < H; ++j)
+                    final_state[((int64_t)s * C + c) * H + j] = (float)XIN(len - H + j);
+#undef XIN
+        }
+    }
+}
+
+/* One-token update for n requests: x [n, C]; state [n_slots, C, W-1] in/out
+ * (the W-1 previous inputs, oldest first); idx [n] slot per request, or NULL
+ * for slot = request; a negative slot is padding (y = 0, no state change). */
+void oracle_conv1d_update(const float* x, const float* w, const float* bias, int W,
+                          float* state, const int32_t* idx, int n, int C, int act, double* y) {
+    const int H = W - 1;
+    for (int r = 0; r < n; ++r) {
+        const int slot = idx ? idx[r] : r;
+        for (int c = 0; c < C; ++c) {
+            if (slot < 0) {
+                y[(int64_t)r * C + c] = 0.0;
+                continue;
+            }
+            float* st = state + ((int64_t)slot * C + c) * H;
+            const double xin = (double)x[(int64_t)r * C + c];
+            double acc = bias ? (double)bias[c] : 0.0;
+            for (int i = 0; i < H; ++i) acc += (double)w[(int64_t)c * W + i] * (double)st[i];
+            acc += (double)w[(int64_t)c * W + H] * xin;
+            y[(int64_t)r * C + c] = act ? silu_f64(acc) : acc;
+            for (int i = 0; i + 1 < H; ++i) st[i] = st[i + 1];
+            if (H > 0) st[H - 1] = x[(int64_t)r * C + c];
+        }
+    }
 }

@@ -26,6 +26,12 @@ MUTANTS = {
     "output_from_key": ("double qi = q[i];", "double qi = k[i];"),
     "softplus_threshold_inclusive": ("(xd > 20.0)", "(xd >= 20.0)"),
     "softplus_log_of_one_plus": ("log1p(exp(xd))", "log(1.0 + exp(xd))"),
+    "conv_taps_reversed": ("acc += (double)w[(int64_t)c * W + i] * XIN(t - H + i);",
+                           "acc += (double)w[(int64_t)c * W + (W - 1 - i)] * XIN(t - H + i);"),
+    "conv_window_shifted": ("acc += (double)w[(int64_t)c * W + i] * XIN(t - H + i);",
+                            "acc += (double)w[(int64_t)c * W + i] * XIN(t - W + i);"),
+    "conv_bias_dropped": ("double acc = bias ? (double)bias[c] : 0.0;\n                for",
+                          "double acc = 0.0;\n                for"),
 }
 
 
@@ -43,6 +49,8 @@ def _build_mutant(tmp_path, name):
     lib.oracle_gdn_fwd.argtypes = [P, P, P, P, P, P, P] + [ctypes.c_int] * 4 + [
         ctypes.c_double, P, P, ctypes.c_int]
     lib.oracle_softplus.argtypes = [P, ctypes.c_int64, P]
+    lib.oracle_conv1d_fwd.argtypes = [P, P, P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P,
+                                      ctypes.c_int, P, P]
     return lib
 
 
@@ -78,13 +86,28 @@ def _softplus_pins_pass(lib):
             and abs(out[3] - math.log1p(math.exp(3.0))) < 1e-15)
 
 
+def _conv_pin_passes(lib):
+    """numpy's convolve on random data, with a bias (pins taps, window, bias)."""
+    rng = np.random.default_rng(5)
+    T, C, W = 11, 3, 4
+    x = rng.standard_normal((T, C)).astype(np.float32)
+    w = rng.standard_normal((C, W)).astype(np.float32)
+    bias = rng.standard_normal(C).astype(np.float32)
+    cu = np.array([0, T], np.int64)
+    y = np.empty((T, C))
+    lib.oracle_conv1d_fwd(_ptr(x), _ptr(w), _ptr(bias), W, _ptr(cu), 1, C, None, 0, _ptr(y), None)
+    ref = np.stack([np.convolve(x[:, c].astype(np.float64), w[c, ::-1].astype(np.float64))[:T]
+                    + bias[c] for c in range(C)], axis=1)
+    return np.allclose(y, ref, rtol=0, atol=1e-12)
+
+
 def test_unmutated_source_passes(tmp_path):
     MUTANTS["identity"] = ("#include <math.h>", "#include <math.h>")
     try:
         lib = _build_mutant(tmp_path, "identity")
     finally:
         del MUTANTS["identity"]
-    assert _recurrence_pin_passes(lib) and _softplus_pins_pass(lib)
+    assert _recurrence_pin_passes(lib) and _softplus_pins_pass(lib) and _conv_pin_passes(lib)
 
 
 @pytest.mark.parametrize("name", ["sign_of_delta", "dropped_beta", "dropped_decay",
@@ -96,3 +119,8 @@ def test_recurrence_mutant_is_caught(tmp_path, name):
 @pytest.mark.parametrize("name", ["softplus_threshold_inclusive", "softplus_log_of_one_plus"])
 def test_softplus_mutant_is_caught(tmp_path, name):
     assert not _softplus_pins_pass(_build_mutant(tmp_path, name))
+
+
+@pytest.mark.parametrize("name", ["conv_taps_reversed", "conv_window_shifted", "conv_bias_dropped"])
+def test_conv_mutant_is_caught(tmp_path, name):
+    assert not _conv_pin_passes(_build_mutant(tmp_path, name))
