@@ -338,6 +338,40 @@ def run_ours(args):
     dby, dfl = decode_algorithmic(dw.n, *dargs)
     dach = dby / (dec_ms * 1e-3) / 1e9
 
+    # --- short convolution (ZzCompute item 1) over the layer's q/k/v channels, and its
+    # one-token update at the decode row width
+    cw = I.CONV_B4_T4096
+    ci = I.conv_inputs(cw)
+    cx, cwt, cb = ci["x"].to(dev), ci["w"].to(dev), ci["bias"].to(dev)
+    cy = torch.empty_like(cx)
+    for _ in range(3):
+        gdn.conv1d_fwd(cx, cwt, cb, activation=True, out=cy)
+    n_cv = max(5, args.steps)
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(n_cv):
+        gdn.conv1d_fwd(cx, cwt, cb, activation=True, out=cy)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    conv_ms = max_over_ranks(c0.elapsed_time(c1), world, dev) / n_cv
+    conv_by = 2 * cx.numel() * cx.element_size() + cwt.numel() * 4 + cb.numel() * 4
+    conv_ach = conv_by / (conv_ms * 1e-3) / 1e9
+    ui = {k: v.to(dev) for k, v in I.conv_decode_inputs(I.CONV_DECODE_N, I.CONV_DECODE_C, cw.W,
+                                                        I.CONV_DECODE_N).items()}
+    uy = torch.empty_like(ui["x"])
+    for _ in range(3):
+        gdn.conv1d_update(ui["x"], ui["w"], ui["conv_state"], ui["bias"], activation=True, out=uy)
+    torch.cuda.synchronize()
+    c0.record(stream)
+    for _ in range(n_cv):
+        gdn.conv1d_update(ui["x"], ui["w"], ui["conv_state"], ui["bias"], activation=True, out=uy)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    upd_ms = max_over_ranks(c0.elapsed_time(c1), world, dev) / n_cv
+    upd_by = (2 * ui["x"].numel() * 2 + 2 * ui["conv_state"].numel() * 2
+              + ui["w"].numel() * 4 + ui["bias"].numel() * 4)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp)
@@ -358,7 +392,7 @@ def run_ours(args):
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "path": "pinned host -> gate_prep -> chunk_fwd -> pinned host (o, h_T)"},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches_per_step * args.steps,  # timed region of the headline step
             "clocks": clk.summary(),
             "decode": {"workload": dw.name, "metric": "requests/s",
                        "value": dw.n * world / (dec_ms * 1e-3), "ms_per_step": dec_ms,
@@ -366,6 +400,16 @@ def run_ours(args):
                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                     "frac": round(dach / peaks["hbm_gbs"], 4),
                                     "algorithmic_bytes": dby}},
+            "conv1d": {"workload": cw.name, "metric": "tokens/s",
+                       "value": cw.B * cw.T * world / (conv_ms * 1e-3), "ms_per_step": conv_ms,
+                       "roofline": {"bound": "hbm", "achieved": round(conv_ach, 1),
+                                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": round(conv_ach / peaks["hbm_gbs"], 4),
+                                    "algorithmic_bytes": conv_by},
+                       "update": {"workload": f"n{I.CONV_DECODE_N} C{I.CONV_DECODE_C} W{cw.W} bf16",
+                                  "ms_per_step": upd_ms,
+                                  "achieved_gbs": round(upd_by / (upd_ms * 1e-3) / 1e9, 1),
+                                  "algorithmic_bytes": upd_by}},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -205,3 +205,73 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
               _ptr(beta), _ptr(h0), _ptr(cu_seqlens), n_seq, B, T, H, K, V, float(scale),
               _ptr(out), _DT[out.dtype], _ptr(hT), int(flags), _stream(q))
     return out, hT
+
+
+def conv1d_fwd(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+               cu_seqlens: Optional[torch.Tensor] = None, init_state: Optional[torch.Tensor] = None,
+               activation: bool = False, final_state: bool = False,
+               out: Optional[torch.Tensor] = None):
+    """Causal depthwise conv1d (ZzCompute item 1): x [B, T, C] (fp32 or bf16), or
+    [1, T_total, C] with cu_seqlens (int32 [n_seq+1]); w [C, W] fp32 (W <= 4); bias
+    [C] fp32; init_state [n_seq, C, W-1] in x's dtype.  Returns y (like x), or
+    (y, final_state [n_seq, C, W-1]) when final_state=True."""
+    _need(x, "x")
+    if x.dtype not in _DT:
+        raise TypeError("x must be float32 or bfloat16")
+    dev = x.device
+    B, T, C = x.shape
+    _need(w, "w", torch.float32, dev)
+    if w.dim() != 2 or w.shape[0] != C:
+        raise ValueError("w must be [C, W]")
+    W = w.shape[1]
+    if bias is not None:
+        _need(bias, "bias", torch.float32, dev)
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if B != 1:
+            raise ValueError("packed sequences need x of shape [1, T_total, C]")
+        n_seq = cu_seqlens.numel() - 1
+    else:
+        n_seq = B
+    if init_state is not None:
+        _need(init_state, "init_state", x.dtype, dev)
+        if tuple(init_state.shape) != (n_seq, C, W - 1):
+            raise ValueError("init_state must be [n_seq, C, W-1]")
+    y = out if out is not None else torch.empty_like(x)
+    _need(y, "out", x.dtype, dev)
+    fin = torch.empty(n_seq, C, max(W - 1, 0), dtype=x.dtype, device=dev) if final_state else None
+    _lib.call("gdn_conv1d_fwd", _ptr(x), _DT[x.dtype], _ptr(w), _ptr(bias), W, _ptr(cu_seqlens),
+              n_seq, B, T, C, _ptr(init_state), _ptr(fin), int(bool(activation)), _ptr(y),
+              _stream(x))
+    return (y, fin) if final_state else y
+
+
+def conv1d_update(x: torch.Tensor, w: torch.Tensor, conv_state: torch.Tensor,
+                  bias: Optional[torch.Tensor] = None, state_idx: Optional[torch.Tensor] = None,
+                  activation: bool = False, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One decode token: x [n, C]; conv_state [n_slots, C, W-1] (updated in place);
+    state_idx int32 [n] (-1 = padding: zero output, state untouched) or None."""
+    _need(x, "x")
+    if x.dtype not in _DT:
+        raise TypeError("x must be float32 or bfloat16")
+    dev = x.device
+    n, C = x.shape
+    _need(w, "w", torch.float32, dev)
+    if w.dim() != 2 or w.shape[0] != C:
+        raise ValueError("w must be [C, W]")
+    W = w.shape[1]
+    _need(conv_state, "conv_state", x.dtype, dev)
+    if conv_state.dim() != 3 or conv_state.shape[1:] != (C, W - 1):
+        raise ValueError("conv_state must be [n_slots, C, W-1]")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, dev)
+    if state_idx is not None:
+        _need(state_idx, "state_idx", torch.int32, dev)
+        if state_idx.numel() != n:
+            raise ValueError("state_idx must have one entry per request")
+    y = out if out is not None else torch.empty_like(x)
+    _need(y, "out", x.dtype, dev)
+    _lib.call("gdn_conv1d_update", _ptr(x), _DT[x.dtype], _ptr(w), _ptr(bias), W,
+              _ptr(conv_state), _ptr(state_idx), n, conv_state.shape[0], C,
+              int(bool(activation)), _ptr(y), _stream(x))
+    return y

@@ -13,6 +13,7 @@
 #include "gates_decode.cuh"
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
+#include "conv1d.cuh"
 
 namespace {
 
@@ -65,6 +66,63 @@ gdn_status launch_simt_dt(const gdn::ChunkArgs& a, gdn_dtype in, gdn_dtype out, 
 constexpr size_t kSimtSmemMax = 227 * 1024;
 
 size_t ws_schedule_bytes(int n_seq) { return ((size_t)n_seq * 4 + 255) / 256 * 256; }
+
+}  // namespace
+
+namespace {
+
+// ------------------------------------------------------------------ conv1d
+
+template <typename T, int NV, int W, bool ACT>
+gdn_status launch_conv_fwd(const gdn::ConvArgs& a, cudaStream_t st) {
+    const int groups = a.C / NV;
+    const int64_t runs = (a.rows + gdn::kConvRun - 1) / gdn::kConvRun;
+    dim3 grid((groups + 127) / 128, (unsigned)(runs < 65535 ? runs : 65535));
+    gdn::conv1d_fwd_kernel<T, NV, W, ACT><<<grid, 128, 0, st>>>(a);
+    return launch_check();
+}
+
+template <typename T, int NV, bool ACT>
+gdn_status conv_fwd_w(const gdn::ConvArgs& a, int W, cudaStream_t st) {
+    switch (W) {
+        case 1: return launch_conv_fwd<T, NV, 1, ACT>(a, st);
+        case 2: return launch_conv_fwd<T, NV, 2, ACT>(a, st);
+        case 3: return launch_conv_fwd<T, NV, 3, ACT>(a, st);
+        default: return launch_conv_fwd<T, NV, 4, ACT>(a, st);
+    }
+}
+
+template <typename T>
+gdn_status conv_fwd_t(const gdn::ConvArgs& a, int W, bool act, bool vec, cudaStream_t st) {
+    constexpr int NV = gdn::ConvVec<T>::N;
+    if (vec) return act ? conv_fwd_w<T, NV, true>(a, W, st) : conv_fwd_w<T, NV, false>(a, W, st);
+    return act ? conv_fwd_w<T, 1, true>(a, W, st) : conv_fwd_w<T, 1, false>(a, W, st);
+}
+
+template <typename T, int NV, int W, bool ACT>
+gdn_status launch_conv_upd(const gdn::ConvUpdateArgs& a, cudaStream_t st) {
+    dim3 grid((a.C / NV + 127) / 128, (unsigned)a.n);
+    gdn::conv1d_update_kernel<T, NV, W, ACT><<<grid, 128, 0, st>>>(a);
+    return launch_check();
+}
+
+template <typename T, int NV, bool ACT>
+gdn_status conv_upd_w(const gdn::ConvUpdateArgs& a, int W, cudaStream_t st) {
+    switch (W) {
+        case 1: return launch_conv_upd<T, NV, 1, ACT>(a, st);
+        case 2: return launch_conv_upd<T, NV, 2, ACT>(a, st);
+        case 3: return launch_conv_upd<T, NV, 3, ACT>(a, st);
+        default: return launch_conv_upd<T, NV, 4, ACT>(a, st);
+    }
+}
+
+template <typename T>
+gdn_status conv_upd_t(const gdn::ConvUpdateArgs& a, int W, bool act, bool vec,
+                             cudaStream_t st) {
+    constexpr int NV = gdn::ConvVec<T>::N;
+    if (vec) return act ? conv_upd_w<T, NV, true>(a, W, st) : conv_upd_w<T, NV, false>(a, W, st);
+    return act ? conv_upd_w<T, 1, true>(a, W, st) : conv_upd_w<T, 1, false>(a, W, st);
+}
 
 }  // namespace
 
@@ -242,6 +300,62 @@ gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, in
     GDN_DEC(32, 128) GDN_DEC(32, 64) GDN_DEC(32, 32)
 #undef GDN_DEC
     return GDN_ERR_UNSUPPORTED;
+}
+
+gdn_status gdn_conv1d_fwd(const void* x, int dtype, const float* w, const float* bias, int W,
+                          const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int C,
+                          const void* init_state, void* final_state, int activation, void* y,
+                          void* stream) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (W < 1 || W > 4 || C < 1 || T < 0 || (activation != 0 && activation != 1))
+        return GDN_ERR_INVALID_ARG;
+    if (cu_seqlens ? (B != 1 || n_seq < 1) : (B < 1 || n_seq != B)) return GDN_ERR_INVALID_ARG;
+    const int64_t rows = cu_seqlens ? T : (int64_t)B * T;
+    if (rows > 0 && (!x || !w || !y || x == y)) return GDN_ERR_INVALID_ARG;
+    if (final_state && final_state == init_state) return GDN_ERR_INVALID_ARG;
+    const size_t es = dtype == GDN_BF16 ? 2 : 4;
+    const int nv = (int)(16 / es);
+    const bool vec = C % nv == 0 && aligned16(x) && aligned16(y) &&
+                     (!init_state || aligned16(init_state)) && (!final_state || aligned16(final_state));
+    gdn::ConvArgs a{x, w, bias, cu_seqlens, n_seq, T, rows, C, init_state, final_state, y};
+    cudaStream_t st = as_stream(stream);
+    if (rows > 0) {
+        gdn_status s = dtype == GDN_BF16
+                           ? conv_fwd_t<__nv_bfloat16>(a, W, activation == 1, vec, st)
+                           : conv_fwd_t<float>(a, W, activation == 1, vec, st);
+        if (s != GDN_OK) return s;
+    }
+    if (final_state && W > 1 && (cu_seqlens || T == 0)) {
+        // empty sequences keep their initial state (or zeros)
+        if (n_seq > 65535) return GDN_ERR_UNSUPPORTED;
+        const int64_t n = (int64_t)C * (W - 1);
+        dim3 grid((unsigned)((n + 255) / 256 < 64 ? (n + 255) / 256 : 64), (unsigned)n_seq);
+        if (dtype == GDN_BF16)
+            gdn::conv1d_final_empty_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a, W - 1);
+        else
+            gdn::conv1d_final_empty_kernel<float><<<grid, 256, 0, st>>>(a, W - 1);
+        return launch_check();
+    }
+    return GDN_OK;
+}
+
+gdn_status gdn_conv1d_update(const void* x, int dtype, const float* w, const float* bias, int W,
+                             void* conv_state, const int32_t* state_idx, int n, int n_slots, int C,
+                             int activation, void* y, void* stream) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (W < 1 || W > 4 || C < 1 || n < 0 || n_slots < 0 || (activation != 0 && activation != 1))
+        return GDN_ERR_INVALID_ARG;
+    if (!state_idx && n_slots < n) return GDN_ERR_INVALID_ARG;
+    if (n == 0) return GDN_OK;
+    if (!x || !w || !y || x == y || (W > 1 && !conv_state)) return GDN_ERR_INVALID_ARG;
+    if (n > 65535) return GDN_ERR_UNSUPPORTED;
+    const size_t es = dtype == GDN_BF16 ? 2 : 4;
+    const int nv = (int)(16 / es);
+    const bool vec = C % nv == 0 && aligned16(x) && aligned16(y);
+    gdn::ConvUpdateArgs a{x, w, bias, conv_state, state_idx, n, n_slots, C, y};
+    cudaStream_t st = as_stream(stream);
+    return dtype == GDN_BF16 ? conv_upd_t<__nv_bfloat16>(a, W, activation == 1, vec, st)
+                             : conv_upd_t<float>(a, W, activation == 1, vec, st);
 }
 
 gdn_status gdn_device_status(void* stream) {

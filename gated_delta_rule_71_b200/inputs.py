@@ -15,6 +15,10 @@ Distributions (shared by all chunked workloads):
   * h0 ~ N(0, 0.1^2) fp32 where a workload has initial states.
 Decode workload: x, ba ~ N(0, 1) bf16; A_log, dt_bias as above; state
 ~ N(0, 0.1^2) fp32.
+Short-convolution workloads (the depthwise conv1d ahead of q/k/v): draws in the
+order x, w, bias, conv state, lengths; x ~ N(0, 1) cast to the workload dtype,
+w ~ N(0, 1/W) fp32 [C, W], bias ~ N(0, 0.1^2) fp32, conv state ~ N(0, 1) in the
+activation dtype.  C = 2*H*K + H*V, the q/k/v channels of a layer.
 """
 from __future__ import annotations
 
@@ -64,6 +68,27 @@ LONG_T131072 = ChunkWorkload("bf16 B1 H32 T131072 K=V=128", 1, 131072, 32, 128, 
 GDP_DECODE = DecodeWorkload("GDP decode n256 M2 H32 G16 P=N=128", 256, 2, 32, 16, 128, 128,
                             seed=1004)
 CHUNK_WORKLOADS = (FP32_SMALL, BF16_B4_T4096, VARLEN_8x32768, LONG_T131072)
+
+
+@dataclass(frozen=True)
+class ConvWorkload:
+    name: str
+    B: int
+    T: int
+    C: int
+    W: int
+    dtype: torch.dtype
+    n_seq_varlen: int = 0      # > 0: packed batch of this many sequences summing to T (B == 1)
+    init_state: bool = False
+    seed: int = 0
+
+
+# The short convolution over the headline layer's q/k/v channels (H=16, K=V=128),
+# and the one-token update on the decode workload's post-conv row width.
+CONV_B4_T4096 = ConvWorkload("conv1d bf16 B4 T4096 C6144 W4 silu", 4, 4096, 6144, 4,
+                             torch.bfloat16, seed=1005)
+CONV_DECODE_N = 256
+CONV_DECODE_C = 2 * 32 * 128 + 2 * 16 * 128 + 16 * 128  # the GDP decode x row (14336)
 
 
 def _normal(gen, shape):
@@ -133,3 +158,31 @@ def decode_inputs(w: DecodeWorkload, seed: Optional[int] = None):
     A_log, dt_bias = _gate_params(gen, H)
     state = _normal(gen, (n, H, N, P)) * 0.1
     return dict(x=x, ba=ba, A_log=A_log, dt_bias=dt_bias, state=state)
+
+
+def conv_inputs(w: ConvWorkload, seed: Optional[int] = None, lengths=None):
+    """x [B, T, C] (or [1, T, C] packed, with cu_seqlens), w [C, W], bias [C], and
+    init_state [n_seq, C, W-1] when the workload has one.  CPU tensors."""
+    gen = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    x = _normal(gen, (w.B, w.T, w.C)).to(w.dtype)
+    wt = _normal(gen, (w.C, w.W)) / math.sqrt(w.W)
+    bias = _normal(gen, (w.C,)) * 0.1
+    n_seq = w.n_seq_varlen if w.n_seq_varlen else w.B
+    init = _normal(gen, (n_seq, w.C, w.W - 1)).to(w.dtype) if w.init_state else None
+    cu = None
+    if w.n_seq_varlen:
+        if lengths is None:
+            lengths = varlen_lengths(gen, w.n_seq_varlen, w.T)
+        cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+    return {"x": x, "w": wt, "bias": bias, "init_state": init, "cu_seqlens": cu}
+
+
+def conv_decode_inputs(n: int, C: int, W: int, n_slots: int, dtype=torch.bfloat16, seed: int = 1006):
+    """x [n, C], w [C, W], bias [C], conv_state [n_slots, C, W-1]."""
+    gen = torch.Generator().manual_seed(seed)
+    x = _normal(gen, (n, C)).to(dtype)
+    wt = _normal(gen, (C, W)) / math.sqrt(W)
+    bias = _normal(gen, (C,)) * 0.1
+    state = _normal(gen, (n_slots, C, W - 1)).to(dtype)
+    return {"x": x, "w": wt, "bias": bias, "conv_state": state}

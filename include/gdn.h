@@ -206,6 +206,54 @@ gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, gd
                                  unsigned flags, void* stream);
 
 /*
+ * gdn_conv1d_fwd -- causal depthwise conv1d over a packed batch (the short
+ * convolution ahead of the gates).
+ * ZzCompute, PyTorch Helion Hackathon gallery entry 11, item 1 ("Causal
+ * Conv1d -- Depthwise Causal Convolution": each channel convolved on its own
+ * with its past context, filter width 4, boundaries by masked loads):
+ *     y[t,c] = bias[c] + sum_{i<W} w[c,i] x[t-(W-1)+i, c],   then y*sigmoid(y)
+ *     when activation == 1 (SiLU),
+ * per sequence; the taps before a sequence's first token read its initial
+ * conv state (its W-1 previous inputs, oldest first) or zero.  Reading: the
+ * last tap w[c,W-1] weighs the current input (the pages give no tap order).
+ *   x, y        [rows, C] of `dtype` (GDN_F32 or GDN_BF16), rows = B*T dense, or
+ *               T (= T_total) with cu_seqlens; y must not overlap x.
+ *   w           [C, W] fp32, 1 <= W <= 4;  bias [C] fp32 or NULL.
+ *   cu_seqlens  NULL: B sequences of T rows (n_seq must equal B); else int32
+ *               [n_seq+1], nondecreasing from 0 to T, B must be 1.
+ *   init_state  [n_seq, C, W-1] of `dtype`, or NULL for zeros.
+ *   final_state [n_seq, C, W-1] of `dtype`, or NULL: each sequence's last W-1
+ *               inputs, oldest first (initial-state values where it is shorter);
+ *               must not be init_state.
+ * Accumulation is fp32 (fmaf, taps in order), one rounding to `dtype`.  All
+ * rows are HBM-streamed once, plus a W-1 row halo per 32-row run.
+ * Returns GDN_ERR_INVALID_ARG for bad sizes/pointers, GDN_ERR_CUDA on launch
+ * failure.
+ */
+gdn_status gdn_conv1d_fwd(const void* x, int dtype, const float* w, const float* bias, int W,
+                          const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int C,
+                          const void* init_state, void* final_state, int activation, void* y,
+                          void* stream);
+
+/*
+ * gdn_conv1d_update -- one decode token through the short convolution.
+ * For request r with slot s = state_idx ? state_idx[r] : r:
+ *     window = [conv_state[s, c, 0..W-2], x[r, c]];  y[r,c] = bias[c] + w[c,:].window
+ *     (SiLU when activation == 1);  conv_state[s, c, :] = window[1..W-1].
+ * A negative slot is padding: y[r,:] = 0 and no state is read or written
+ * (Megatron-Core "core.ssm.ops.gdp.decode_prepare", module description: "a -1
+ * slot zeroes its conv output").  A slot >= n_slots is treated the same way and
+ * records GDN_ERR_INVALID_ARG in the device status word.
+ *   x, y        [n, C] of `dtype`; y must not overlap x.
+ *   conv_state  [n_slots, C, W-1] of `dtype`, in place; may be NULL when W == 1.
+ *   state_idx   int32 [n] or NULL (then n_slots >= n and slot = r).  Distinct
+ *               requests must name distinct slots.
+ */
+gdn_status gdn_conv1d_update(const void* x, int dtype, const float* w, const float* bias, int W,
+                             void* conv_state, const int32_t* state_idx, int n, int n_slots, int C,
+                             int activation, void* y, void* stream);
+
+/*
  * gdn_device_status -- reads and clears the device status word on the current
  * device.  Kernels that wait on the device (mbarrier waits in the tensor-core
  * kernel) give up after a bounded number of polls, record GDN_ERR_TIMEOUT

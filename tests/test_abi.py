@@ -107,3 +107,31 @@ def test_package_has_no_cpu_fallback():
         if fn.endswith(".py"):
             src = open(os.path.join(pkg, fn)).read()
             assert "import oracle" not in src and "from oracle" not in src, fn
+
+
+def test_conv1d_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    q = ctypes.c_void_p(512)
+
+    def fwd(x=p, dt=1, w=p, W=4, cu=None, n_seq=2, B=2, T=8, C=16, init=None, fin=None, act=0,
+            y=q):
+        return lib.gdn_conv1d_fwd(x, dt, w, None, W, cu, n_seq, B, T, C, init, fin, act, y, None)
+
+    assert fwd(dt=3) == INVALID
+    assert fwd(W=0) == INVALID and fwd(W=5) == INVALID
+    assert fwd(C=0) == INVALID and fwd(T=-1) == INVALID
+    assert fwd(act=2) == INVALID
+    assert fwd(n_seq=3) == INVALID                 # dense: n_seq must equal B
+    assert fwd(cu=p, n_seq=2, B=2) == INVALID      # packed: B must be 1
+    assert fwd(x=None) == INVALID and fwd(y=p) == INVALID  # y may not alias x
+    assert fwd(init=q, fin=q) == INVALID
+
+    def upd(x=p, dt=0, W=4, st=q, idx=None, n=4, n_slots=4, C=16, act=0, y=ctypes.c_void_p(768)):
+        return lib.gdn_conv1d_update(x, dt, p, None, W, st, idx, n, n_slots, C, act, y, None)
+
+    assert upd(n_slots=3) == INVALID               # no index: every request needs its slot
+    assert upd(st=None) == INVALID
+    assert upd(n=-1) == INVALID and upd(W=9) == INVALID
+    assert upd(y=p) == INVALID
+    assert upd(n=0) == 0                           # nothing to do
