@@ -39,7 +39,7 @@ struct ConvArgs {
     void* y;
 };
 
-constexpr int kConvRun = 32;   // rows per thread
+constexpr int kConvRun = 64;   // rows per thread
 constexpr int kConvBatch = 8;  // rows loaded ahead of use
 
 template <typename T> struct ConvVec { static constexpr int N = 16 / sizeof(T); };
@@ -118,7 +118,7 @@ __device__ __forceinline__ void conv_find_seq(const ConvArgs& a, int64_t r, int&
 // kConvRun rows (grid-stride).  A run may cross sequence boundaries: the window
 // restarts from the next sequence's initial state there.
 template <typename T, int NV, int W, bool ACT>
-__global__ void __launch_bounds__(128) conv1d_fwd_kernel(const ConvArgs a) {
+__global__ void __launch_bounds__(128, 4) conv1d_fwd_kernel(const ConvArgs a) {
     constexpr int H = W - 1;
     const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * NV;
     if (c0 >= a.C) return;
@@ -236,45 +236,83 @@ struct ConvUpdateArgs {
     void* y;             // [n, C]
 };
 
-// Grid: x over groups of NV channels (128 threads per block), y over requests.
-// Requests must name distinct slots (each slot's window is read and written by
-// the threads of one request).
+constexpr int kConvReqs = 8;  // requests per thread in the update (weights loaded once)
+
+// Grid: x over groups of NV channels (128 threads per block), y over groups of
+// kConvReqs requests.  Requests must name distinct slots (each slot's window is
+// read and written by the threads of one request).
 template <typename T, int NV, int W, bool ACT>
 __global__ void __launch_bounds__(128) conv1d_update_kernel(const ConvUpdateArgs a) {
     constexpr int H = W - 1;
     const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * NV;
-    const int r = blockIdx.y;
     if (c0 >= a.C) return;
     const T* x = static_cast<const T*>(a.x);
     T* y = static_cast<T*>(a.y);
     T* state = static_cast<T*>(a.state);
-    const int slot = a.idx ? a.idx[r] : r;
-    float o[NV];
-    if (slot < 0 || slot >= a.n_slots) {
-        if (slot >= a.n_slots) record_status(GDN_ERR_INVALID_ARG);
-#pragma unroll
-        for (int j = 0; j < NV; ++j) o[j] = 0.f;
-        conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
-        return;
-    }
-    float xc[NV];
-    conv_load<T, NV>(x + (int64_t)r * a.C + c0, xc);
-    T* sp = state + ((int64_t)slot * a.C + c0) * H;
+    float wt[W][NV], bs[NV];
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
-        float win[H > 0 ? H : 1];
 #pragma unroll
-        for (int i = 0; i < H; ++i) win[i] = to_f32(sp[j * H + i]);
-        float acc = a.bias ? a.bias[c0 + j] : 0.f;
-#pragma unroll
-        for (int i = 0; i < H; ++i) acc = fmaf(a.w[(int64_t)(c0 + j) * W + i], win[i], acc);
-        acc = fmaf(a.w[(int64_t)(c0 + j) * W + H], xc[j], acc);
-        o[j] = ACT ? conv_silu(acc) : acc;
-#pragma unroll
-        for (int i = 0; i + 1 < H; ++i) sp[j * H + i] = from_f32<T>(win[i + 1]);
-        if constexpr (H > 0) sp[j * H + H - 1] = from_f32<T>(xc[j]);
+        for (int i = 0; i < W; ++i) wt[i][j] = a.w[(int64_t)(c0 + j) * W + i];
+        bs[j] = a.bias ? a.bias[c0 + j] : 0.f;
     }
-    conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
+    const int rend = (blockIdx.y + 1) * kConvReqs < a.n ? (blockIdx.y + 1) * kConvReqs : a.n;
+    for (int r = blockIdx.y * kConvReqs; r < rend; ++r) {
+        const int slot = a.idx ? a.idx[r] : r;
+        float o[NV];
+        if (slot < 0 || slot >= a.n_slots) {
+            if (slot >= a.n_slots) record_status(GDN_ERR_INVALID_ARG);
+#pragma unroll
+            for (int j = 0; j < NV; ++j) o[j] = 0.f;
+            conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
+            continue;
+        }
+        float xc[NV];
+        conv_load<T, NV>(x + (int64_t)r * a.C + c0, xc);
+        T* sp = state + ((int64_t)slot * a.C + c0) * H;  // NV*H contiguous values
+        if constexpr (NV * sizeof(T) == 16) {
+            // the window is H 16-byte units; element e = j*H + i sits in unit e / NV
+            uint4 wu[H > 0 ? H : 1], nu[H > 0 ? H : 1];
+#pragma unroll
+            for (int u = 0; u < H; ++u) wu[u] = reinterpret_cast<const uint4*>(sp)[u];
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                float acc = bs[j];
+#pragma unroll
+                for (int i = 0; i < H; ++i) {
+                    const int e = j * H + i;
+                    acc = fmaf(wt[i][j], to_f32(reinterpret_cast<const T*>(&wu[e / NV])[e % NV]), acc);
+                }
+                acc = fmaf(wt[H][j], xc[j], acc);
+                o[j] = ACT ? conv_silu(acc) : acc;
+#pragma unroll
+                for (int i = 0; i < H; ++i) {
+                    const int e = j * H + i;
+                    const T v = (i + 1 < H) ? reinterpret_cast<const T*>(&wu[(e + 1) / NV])[(e + 1) % NV]
+                                            : from_f32<T>(xc[j]);
+                    reinterpret_cast<T*>(&nu[e / NV])[e % NV] = v;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < H; ++u) reinterpret_cast<uint4*>(sp)[u] = nu[u];
+        } else {
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                float win[H > 0 ? H : 1];
+#pragma unroll
+                for (int i = 0; i < H; ++i) win[i] = to_f32(sp[j * H + i]);
+                float acc = bs[j];
+#pragma unroll
+                for (int i = 0; i < H; ++i) acc = fmaf(wt[i][j], win[i], acc);
+                acc = fmaf(wt[H][j], xc[j], acc);
+                o[j] = ACT ? conv_silu(acc) : acc;
+#pragma unroll
+                for (int i = 0; i + 1 < H; ++i) sp[j * H + i] = from_f32<T>(win[i + 1]);
+                if constexpr (H > 0) sp[j * H + H - 1] = from_f32<T>(xc[j]);
+            }
+        }
+        conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
+    }
 }
 
 }  // namespace gdn

@@ -101,7 +101,7 @@ gdn_status conv_fwd_t(const gdn::ConvArgs& a, int W, bool act, bool vec, cudaStr
 
 template <typename T, int NV, int W, bool ACT>
 gdn_status launch_conv_upd(const gdn::ConvUpdateArgs& a, cudaStream_t st) {
-    dim3 grid((a.C / NV + 127) / 128, (unsigned)a.n);
+    dim3 grid((a.C / NV + 127) / 128, (unsigned)((a.n + gdn::kConvReqs - 1) / gdn::kConvReqs));
     gdn::conv1d_update_kernel<T, NV, W, ACT><<<grid, 128, 0, st>>>(a);
     return launch_check();
 }
@@ -348,10 +348,11 @@ gdn_status gdn_conv1d_update(const void* x, int dtype, const float* w, const flo
     if (!state_idx && n_slots < n) return GDN_ERR_INVALID_ARG;
     if (n == 0) return GDN_OK;
     if (!x || !w || !y || x == y || (W > 1 && !conv_state)) return GDN_ERR_INVALID_ARG;
-    if (n > 65535) return GDN_ERR_UNSUPPORTED;
+    if (n > 65535 * gdn::kConvReqs) return GDN_ERR_UNSUPPORTED;
     const size_t es = dtype == GDN_BF16 ? 2 : 4;
     const int nv = (int)(16 / es);
-    const bool vec = C % nv == 0 && aligned16(x) && aligned16(y);
+    const bool vec = C % nv == 0 && aligned16(x) && aligned16(y) &&
+                     (!conv_state || aligned16(conv_state));
     gdn::ConvUpdateArgs a{x, w, bias, conv_state, state_idx, n, n_slots, C, y};
     cudaStream_t st = as_stream(stream);
     return dtype == GDN_BF16 ? conv_upd_t<__nv_bfloat16>(a, W, activation == 1, vec, st)

@@ -226,7 +226,7 @@ gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, gd
  *               inputs, oldest first (initial-state values where it is shorter);
  *               must not be init_state.
  * Accumulation is fp32 (fmaf, taps in order), one rounding to `dtype`.  All
- * rows are HBM-streamed once, plus a W-1 row halo per 32-row run.
+ * rows are HBM-streamed once, plus a W-1 row halo per 64-row run.
  * Returns GDN_ERR_INVALID_ARG for bad sizes/pointers, GDN_ERR_CUDA on launch
  * failure.
  */

@@ -78,8 +78,8 @@ def test_no_activation_no_init(cuda_device):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_varlen_edge_lengths(cuda_device, dtype):
-    # lengths around the 32-row run and the W-1 halo, and empty sequences
-    lens = [1, 2, 3, 0, 4, 31, 32, 33, 0, 63, 64, 65, 5]
+    # lengths around the 64-row run and the W-1 halo, and empty sequences
+    lens = [1, 2, 3, 0, 4, 31, 32, 33, 0, 63, 64, 65, 5, 127, 128, 129, 2]
     wl = I.ConvWorkload("t", 1, sum(lens), 24, 4, dtype, n_seq_varlen=len(lens), init_state=True,
                         seed=13)
     y, fin, ry, rfin, S = _run_fwd(cuda_device, wl, lengths=lens)
