@@ -64,10 +64,15 @@ def decode_algorithmic(n, M, H, G, P, N):
     return by, fl
 
 
-def kernel_source_sha():
+# Sources the tensor-core chunk kernel is built from: a committed ncu summary
+# stays valid while these are unchanged.
+CHUNK_KERNEL_SOURCES = ("chunk_tc.cuh", "tc_ptx.cuh", "common.cuh", "chunk_simt.cuh")
+
+
+def kernel_source_sha(files=CHUNK_KERNEL_SOURCES):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_71_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(files):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
