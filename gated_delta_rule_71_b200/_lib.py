@@ -27,6 +27,8 @@ SIGNATURES = {
                                  P, P]),
     "gdp_decode_step": (I32, [P, I64, P, I64, P, P, I32, I32, I32, I32, I32, I32, P, P, F32, I32,
                               P]),
+    "gdp_decode_step_indexed": (I32, [P, I64, P, I64, P, P, I32, I32, I32, I32, I32, I32, P, P,
+                                      I32, P, F32, I32, P]),
     "gdn_chunk_fwd_noalloc": (I32, [P, P, P, I32, P, P, P, P, I32, I32, I64, I32, I32, I32, F32,
                                     P, I32, P, U32, P]),
     "gdn_conv1d_fwd": (I32, [P, I32, P, P, I32, P, I32, I32, I64, I32, P, P, I32, P, P]),

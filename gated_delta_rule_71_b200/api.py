@@ -153,17 +153,33 @@ def gdp_decode_prepare(x, ba, A_log, dt_bias, M, H, G, P, N):
 
 
 def gdp_decode_step(x, ba, A_log, dt_bias, state, M, H, G, P, N, scale=1.0, qk_l2norm=True,
-                    out=None):
-    """Fused decode step; updates state [n,H,N,P] fp32 in place, returns o [n,H,P] bf16."""
+                    out=None, state_indices=None):
+    """Fused decode step; returns o [n,H,P] bf16 and updates the state in place.
+
+    Without state_indices, state is [n,H,N,P] and request r owns state[r].  With
+    state_indices (int32 [n] on the device), state is a pool [n_slots,H,N,P],
+    request r owns state[state_indices[r]], and a negative index marks a padding
+    request (o = 0, no state touched)."""
     dev, n, xs, bas = _decode_common(x, ba, A_log, dt_bias, M, H, G, P, N)
     _need(state, "state", torch.float32, dev)
-    if tuple(state.shape) != (n, H, N, P):
-        raise ValueError("state must be [n, H, N, P]")
+    if state.dim() != 4 or tuple(state.shape[1:]) != (H, N, P):
+        raise ValueError("state must be [n_slots, H, N, P]")
     if out is None:
         out = torch.empty((n, H, P), dtype=torch.bfloat16, device=dev)
     _need(out, "out", torch.bfloat16, dev)
-    _lib.call("gdp_decode_step", _ptr(x), xs, _ptr(ba), bas, _ptr(A_log), _ptr(dt_bias), n, M, H,
-              G, P, N, _ptr(state), _ptr(out), float(scale), int(bool(qk_l2norm)), _stream(x))
+    if state_indices is None:
+        if state.shape[0] != n:
+            raise ValueError("state must be [n, H, N, P] without state_indices")
+        _lib.call("gdp_decode_step", _ptr(x), xs, _ptr(ba), bas, _ptr(A_log), _ptr(dt_bias), n,
+                  M, H, G, P, N, _ptr(state), _ptr(out), float(scale), int(bool(qk_l2norm)),
+                  _stream(x))
+    else:
+        _need(state_indices, "state_indices", torch.int32, dev)
+        if tuple(state_indices.shape) != (n,):
+            raise ValueError("state_indices must be int32 [n]")
+        _lib.call("gdp_decode_step_indexed", _ptr(x), xs, _ptr(ba), bas, _ptr(A_log),
+                  _ptr(dt_bias), n, M, H, G, P, N, _ptr(state), _ptr(state_indices),
+                  int(state.shape[0]), _ptr(out), float(scale), int(bool(qk_l2norm)), _stream(x))
     return out
 
 

@@ -76,8 +76,13 @@ __global__ void __launch_bounds__(256) gdp_prepare_kernel(
 }
 
 // ---------------------------------------------------------------- decode step
-// One block (8 warps) per (request, head).  The fp32 state [N, P] lives in
-// registers: warp w owns key rows [w*N/8, (w+1)*N/8), lane l owns value
+// One block (8 warps) per (request, head).  The request's state sits in slot
+// state_idx[r] of the state pool (slot r when state_idx is NULL); a negative
+// slot is a padding request: o = 0 and its state is neither read nor written
+// (Megatron-Core "core.ssm.ops.gdp.decode_prepare", module description: the
+// batch is padded upstream with -1 slots).  A slot >= n_slots is handled the
+// same way and records GDN_ERR_INVALID_ARG in the device status word.  The
+// fp32 state [N, P] lives in registers: warp w owns key rows [w*N/8, (w+1)*N/8), lane l owns value
 // columns [l*P/32, (l+1)*P/32), so every row is read and written as one
 // coalesced 512-byte (P = 128) warp access.  Column reductions over the key
 // axis go through shared memory.  The state is read once and written once:
@@ -89,7 +94,8 @@ template <int N, int P>
 __global__ void __launch_bounds__(256) gdp_step_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t xs, const __nv_bfloat16* __restrict__ ba,
     int64_t bas, const float* __restrict__ A_log, const float* __restrict__ dt_bias, int M, int H,
-    int G, float* __restrict__ state, __nv_bfloat16* __restrict__ o, float scale, int l2) {
+    int G, float* __restrict__ state, const int32_t* __restrict__ state_idx, int n_slots,
+    __nv_bfloat16* __restrict__ o, float scale, int l2) {
     constexpr int RPW = N / kDecWarps;  // rows per warp
     constexpr int CPL = P / 32;         // columns per lane
     __shared__ float kv[kDecMaxM][N];
@@ -107,9 +113,15 @@ __global__ void __launch_bounds__(256) gdp_step_kernel(
     const __nv_bfloat16* xr = x + (int64_t)r * xs;
     const __nv_bfloat16* br = ba + (int64_t)r * bas;
     const int64_t kbase = (int64_t)M * H * P, qbase = kbase + (int64_t)M * G * N;
+    const int slot = state_idx ? state_idx[r] : r;
+    if (slot < 0 || slot >= n_slots) {  // padding (uniform across the block)
+        if (slot >= n_slots && threadIdx.x == 0) record_status(GDN_ERR_INVALID_ARG);
+        if (threadIdx.x < P) o[(int64_t)rh * P + threadIdx.x] = __float2bfloat16_rn(0.f);
+        return;
+    }
 
     // 1. issue the state loads first (the only large traffic)
-    float* st = state + (int64_t)rh * N * P;
+    float* st = state + ((int64_t)slot * H + h) * N * P;
     float s[RPW][CPL];
 #pragma unroll
     for (int rr = 0; rr < RPW; ++rr) {

@@ -275,14 +275,17 @@ gdn_status gdp_decode_prepare(const void* x, int64_t x_n_stride, const void* ba,
     return launch_check();
 }
 
-gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, int64_t ba_n_stride,
-                           const float* A_log, const float* dt_bias, int n, int M, int H, int G,
-                           int P, int N, float* state, void* o, float scale, int qk_l2norm,
-                           void* stream) {
+gdn_status gdp_decode_step_indexed(const void* x, int64_t x_n_stride, const void* ba,
+                                   int64_t ba_n_stride, const float* A_log, const float* dt_bias,
+                                   int n, int M, int H, int G, int P, int N, float* state,
+                                   const int32_t* state_idx, int n_slots, void* o, float scale,
+                                   int qk_l2norm, void* stream) {
     gdn_status s = decode_args_ok(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P, N);
     if (s != GDN_OK) return s;
     if (n == 0) return GDN_OK;
-    if (!state || !o || !aligned16(state)) return GDN_ERR_INVALID_ARG;
+    if (!o || n_slots < 0 || (!state_idx && n_slots < n)) return GDN_ERR_INVALID_ARG;
+    if (n_slots > 0 && (!state || !aligned16(state))) return GDN_ERR_INVALID_ARG;
+    if (state_idx && (reinterpret_cast<uintptr_t>(state_idx) & 3u)) return GDN_ERR_INVALID_ARG;
     if (M > gdn::kDecMaxM) return GDN_ERR_UNSUPPORTED;
     if ((int64_t)n * H > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
     using bf = __nv_bfloat16;
@@ -292,7 +295,8 @@ gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, in
     if (N == NN && P == PP) {                                                                    \
         gdn::gdp_step_kernel<NN, PP><<<nb, 256, 0, st>>>((const bf*)x, x_n_stride, (const bf*)ba, \
                                                           ba_n_stride, A_log, dt_bias, M, H, G,  \
-                                                          state, (bf*)o, scale, qk_l2norm);      \
+                                                          state, state_idx, n_slots, (bf*)o,     \
+                                                          scale, qk_l2norm);                     \
         return launch_check();                                                                   \
     }
     GDN_DEC(128, 128) GDN_DEC(128, 64) GDN_DEC(128, 32)
@@ -300,6 +304,15 @@ gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, in
     GDN_DEC(32, 128) GDN_DEC(32, 64) GDN_DEC(32, 32)
 #undef GDN_DEC
     return GDN_ERR_UNSUPPORTED;
+}
+
+gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, int64_t ba_n_stride,
+                           const float* A_log, const float* dt_bias, int n, int M, int H, int G,
+                           int P, int N, float* state, void* o, float scale, int qk_l2norm,
+                           void* stream) {
+    if (n > 0 && !state) return GDN_ERR_INVALID_ARG;
+    return gdp_decode_step_indexed(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P,
+                                   N, state, nullptr, n, o, scale, qk_l2norm, stream);
 }
 
 gdn_status gdn_conv1d_fwd(const void* x, int dtype, const float* w, const float* bias, int W,

@@ -174,6 +174,29 @@ gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, in
                            void* stream);
 
 /*
+ * gdp_decode_step_indexed -- gdp_decode_step on a pool of states.  Request r
+ * uses state slot s = state_idx ? state_idx[r] : r of `state`.
+ *   state     : fp32 [n_slots, H, N, P], the slots named by state_idx read and
+ *               written in place (others untouched); may be NULL when
+ *               n_slots == 0 (every request padding).
+ *   state_idx : int32 [n] device array, or NULL (then n_slots >= n).  Distinct
+ *               requests must name distinct slots (two requests on one slot
+ *               race).  No host read: the call stays graph-capturable.
+ * A negative slot is a padding request: o[r] = 0 and no state is read or
+ * written (Megatron-Core "core.ssm.ops.gdp.decode_prepare", module
+ * description: the batch is padded upstream, with -1 slots).  A slot >=
+ * n_slots is treated the same way and records GDN_ERR_INVALID_ARG in the
+ * device status word (read by gdn_device_status).
+ * Other arguments and errors as gdp_decode_step; also INVALID_ARG for
+ * n_slots < 0, state_idx == NULL with n_slots < n, a misaligned state_idx.
+ */
+gdn_status gdp_decode_step_indexed(const void* x, int64_t x_n_stride, const void* ba,
+                                   int64_t ba_n_stride, const float* A_log, const float* dt_bias,
+                                   int n, int M, int H, int G, int P, int N, float* state,
+                                   const int32_t* state_idx, int n_slots, void* o, float scale,
+                                   int qk_l2norm, void* stream);
+
+/*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate
  * device memory.  The sources describe no such entry point; it exists because
  * some callers have no way to provide the packed-batch workspace: code running

@@ -195,6 +195,31 @@ def gdp_decode_step(x, ba, A_log, dt_bias, state, M, H, G, P, N, scale=1.0, qk_l
     return o, st_out
 
 
+def gdp_decode_step_indexed(x, ba, A_log, dt_bias, state_pool, state_idx, M, H, G, P, N,
+                            scale=1.0, qk_l2norm=True):
+    """Decode step on a pool of states: request r uses slot state_idx[r]; a
+    negative slot is a padding request (Megatron-Core
+    "core.ssm.ops.gdp.decode_prepare", module description: the batch is padded
+    upstream with -1 slots): its output is 0 and no state is touched.  The
+    other requests run gdp_decode_step from their slot's state.
+    Returns (o [n, H, P] fp64, new pool [n_slots, H, N, P] fp64)."""
+    idx = state_idx.cpu().numpy() if hasattr(state_idx, "cpu") else np.asarray(state_idx)
+    idx = idx.astype(np.int64)
+    pool = np.array(_f32(state_pool), dtype=np.float64, copy=True)
+    n = idx.shape[0]
+    o = np.zeros((n, H, P), np.float64)
+    live = np.nonzero(idx >= 0)[0]
+    if live.size:
+        xs = x[live] if hasattr(x, "shape") else x
+        bs = ba[live] if hasattr(ba, "shape") else ba
+        st = _f32(state_pool)[idx[live]]
+        ol, sl = gdp_decode_step(xs, bs, A_log, dt_bias, st, M, H, G, P, N, scale=scale,
+                                 qk_l2norm=qk_l2norm)
+        o[live] = ol
+        pool[idx[live]] = sl
+    return o, pool
+
+
 def conv1d_fwd(x, w, bias=None, cu_seqlens=None, init_state=None, activation=False):
     """Causal depthwise conv1d in fp64.
 

@@ -94,6 +94,14 @@ def test_decode_rejects_bad_arguments():
     big = [p, 9 * H * P + 9 * G * N + G * N, p, 9 * H + H, p, p, n, 9, H, G, P, N]
     assert lib.gdp_decode_step(*big, p, p, 1.0, 1, None) == UNSUPPORTED  # M > 8
     assert lib.gdp_decode_step(*ok[:6], 0, *ok[7:], p, p, 1.0, 1, None) == 0  # n == 0
+    # pooled states: (state, state_idx, n_slots, o, scale, qk_l2norm, stream)
+    ix = lib.gdp_decode_step_indexed
+    assert ix(*ok, p, p, -1, p, 1.0, 1, None) == INVALID                  # n_slots < 0
+    assert ix(*ok, p, None, n - 1, p, 1.0, 1, None) == INVALID            # no index, pool < n
+    assert ix(*ok, p, ctypes.c_void_p(258), n, p, 1.0, 1, None) == INVALID  # misaligned index
+    assert ix(*ok, None, p, 8, p, 1.0, 1, None) == INVALID                # no pool
+    assert ix(*ok, p, p, 8, None, 1.0, 1, None) == INVALID                # no output
+    assert ix(*big, p, p, 8, p, 1.0, 1, None) == UNSUPPORTED              # M > 8
 
 
 def test_selftest_rejects_zero_polls():

@@ -289,3 +289,34 @@ def test_decode_step_is_the_rule_over_the_copies(l2):
         tol = 1e-6 if l2 else 1e-12
         np.testing.assert_allclose(o[r], ofw[0, -1], rtol=0, atol=tol)
         np.testing.assert_allclose(st[r], hT[0], rtol=0, atol=tol)
+
+
+def test_decode_indexed_padding_and_slots():
+    # a pool of states addressed by slot: identity slots reproduce the plain step,
+    # a permutation permutes it, and a -1 slot is a padding request (o = 0, no
+    # state touched)
+    n, M, H, G, P, N = 4, 2, 2, 1, 8, 8
+    gen = torch.Generator().manual_seed(21)
+    x = torch.randn(n, 1, M * H * P + M * G * N + G * N, generator=gen).to(torch.bfloat16)
+    ba = torch.randn(n, 1, M * H + H, generator=gen).to(torch.bfloat16)
+    A_log = torch.rand(H, generator=gen)
+    dt_bias = torch.randn(H, generator=gen)
+    pool = torch.randn(6, H, N, P, generator=gen) * 0.1
+    o_ref, st_ref = oracle.gdp_decode_step(x, ba, A_log, dt_bias, pool[:n], M, H, G, P, N)
+    o, new = oracle.gdp_decode_step_indexed(x, ba, A_log, dt_bias, pool, np.arange(n), M, H, G,
+                                            P, N)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(new[:n], st_ref)
+    np.testing.assert_array_equal(new[n:], pool[n:].double().numpy())
+    perm = np.array([5, 2, -1, 0])
+    o, new = oracle.gdp_decode_step_indexed(x, ba, A_log, dt_bias, pool, perm, M, H, G, P, N)
+    assert (o[2] == 0).all()
+    for r, sl in enumerate(perm):
+        if sl < 0:
+            continue
+        o1, s1 = oracle.gdp_decode_step(x[r:r + 1], ba[r:r + 1], A_log, dt_bias, pool[sl][None],
+                                        M, H, G, P, N)
+        np.testing.assert_array_equal(o[r], o1[0])
+        np.testing.assert_array_equal(new[sl], s1[0])
+    for sl in (1, 3, 4):  # slots no request names are untouched
+        np.testing.assert_array_equal(new[sl], pool[sl].double().numpy())
