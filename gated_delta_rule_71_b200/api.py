@@ -183,6 +183,53 @@ def gdp_decode_step(x, ba, A_log, dt_bias, state, M, H, G, P, N, scale=1.0, qk_l
     return out
 
 
+def gdp_prefill_workspace_size(n_seq, rows, M, H, P, N, o_dtype=torch.float32, packed=False):
+    return int(_lib.load().gdp_prefill_workspace_size(n_seq, rows, M, H, P, N, _DT[o_dtype],
+                                                      int(bool(packed))))
+
+
+def gdp_prefill(x, ba, A_log, dt_bias, M, H, G, P, N, h0=None, cu_seqlens=None, scale=1.0,
+                o_dtype=torch.float32, output_final_state=True, workspace=None):
+    """Gated Delta Product over a prompt.  x [B,T,M*H*P+M*G*N+G*N] and
+    ba [B,T,M*H+H] bf16 rows in the decode layout (B == 1 with cu_seqlens);
+    h0 [n_seq,H,N,P] fp32 or None.  Returns (o [B,T,H,P] in o_dtype, hT
+    [n_seq,H,N,P] fp32 or None): the rule over every token's M copies, o at
+    each token's last copy."""
+    dev = x.device
+    _need(x, "x", torch.bfloat16, dev, contiguous=False)
+    _need(ba, "ba", torch.bfloat16, dev, contiguous=False)
+    if x.dim() != 3 or ba.dim() != 3 or x.shape[:2] != ba.shape[:2]:
+        raise ValueError("x and ba must be [B, T, *] with the same B, T")
+    B, T = int(x.shape[0]), int(x.shape[1])
+    x2, ba2 = x.reshape(B * T, x.shape[2]), ba.reshape(B * T, ba.shape[2])
+    if x2.stride(1) != 1 or ba2.stride(1) != 1:
+        raise ValueError("x and ba rows must be contiguous in their last dimension")
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias")):
+        _need(t, n, torch.float32, dev)
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if B != 1:
+            raise ValueError("packed sequences need B == 1")
+        n_seq = cu_seqlens.numel() - 1
+    else:
+        n_seq = B
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, dev)
+        if tuple(h0.shape) != (n_seq, H, N, P):
+            raise ValueError("h0 must be [n_seq, H, N, P]")
+    o = torch.empty((B, T, H, P), dtype=o_dtype, device=dev)
+    hT = torch.empty((n_seq, H, N, P), dtype=torch.float32, device=dev) if output_final_state \
+        else None
+    need = gdp_prefill_workspace_size(n_seq, B * T, M, H, P, N, o_dtype, cu_seqlens is not None)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _lib.call("gdp_prefill", _ptr(x2), x2.stride(0), _ptr(ba2), ba2.stride(0), _ptr(A_log),
+              _ptr(dt_bias), _ptr(h0), _ptr(cu_seqlens), n_seq, B, T, M, H, G, P, N,
+              float(scale), _ptr(o), _DT[o_dtype], _ptr(hT), _ptr(workspace),
+              workspace.numel() * workspace.element_size(), _stream(x))
+    return o, hT
+
+
 def device_status(device=None) -> int:
     """Reads and clears the device status word (synchronises the current stream)."""
     s = torch.cuda.current_stream(device).cuda_stream

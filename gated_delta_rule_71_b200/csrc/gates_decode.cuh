@@ -241,3 +241,31 @@ __global__ void __launch_bounds__(256) gdp_step_kernel(
 }
 
 }  // namespace gdn
+
+namespace gdn {
+
+// --------------------------------------------------------------- GDP prefill
+// The prefill runs the rule over the copy-interleaved sequence that
+// gdp_decode_prepare builds from T token rows (T*M rows, copy-minor), so the
+// packed-batch offsets scale by M and each token's output is the one at its
+// last copy.
+__global__ void gdp_scale_offsets_kernel(const int32_t* __restrict__ cu, int n, int M,
+                                         int32_t* __restrict__ out) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= n; i += gridDim.x * blockDim.x)
+        out[i] = cu[i] * M;
+}
+
+// o[r] = o_all[r*M + M-1] for rows of `row_units` 16-byte units.
+__global__ void __launch_bounds__(256) gdp_last_copy_kernel(const uint4* __restrict__ o_all,
+                                                            int64_t rows, int M,
+                                                            int64_t row_units,
+                                                            uint4* __restrict__ o) {
+    const int64_t total = rows * row_units;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / row_units, u = i - r * row_units;
+        o[i] = o_all[(r * M + M - 1) * row_units + u];
+    }
+}
+
+}  // namespace gdn

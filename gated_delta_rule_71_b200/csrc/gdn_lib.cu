@@ -315,6 +315,100 @@ gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, in
                                    N, state, nullptr, n, o, scale, qk_l2norm, stream);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------- GDP prefill
+
+namespace {
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+struct PrefillLayout {
+    size_t q, k, v, beta, g, o_all, cu, chunk, total;
+};
+
+PrefillLayout prefill_layout(int n_seq, int64_t rows, int M, int H, int P, int N, gdn_dtype odt,
+                             bool packed) {
+    PrefillLayout L;
+    const size_t cr = (size_t)rows * M * H;  // copy rows x heads
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t at = off; off += align256(bytes); return at; };
+    L.q = take(cr * N * 2);
+    L.k = take(cr * N * 2);
+    L.v = take(cr * P * 2);
+    L.beta = take(cr * 4);
+    L.g = take(cr * 4);
+    L.o_all = take(cr * P * (odt == GDN_BF16 ? 2 : 4));
+    L.cu = packed ? take((size_t)(n_seq + 1) * 4) : off;
+    L.chunk = off;
+    off += packed ? align256(gdn_chunk_fwd_workspace_size(n_seq, rows * M, H, N, P, GDN_BF16)) : 0;
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdp_prefill_workspace_size(int n_seq, int64_t rows, int M, int H, int P, int N,
+                                  gdn_dtype o_dtype, int packed) {
+    if (n_seq < 0 || rows < 0 || M < 1 || H < 1 || P < 1 || N < 1) return 0;
+    return prefill_layout(n_seq, rows, M, H, P, N, o_dtype, packed != 0).total;
+}
+
+gdn_status gdp_prefill(const void* x, int64_t x_n_stride, const void* ba, int64_t ba_n_stride,
+                       const float* A_log, const float* dt_bias, const float* h0,
+                       const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int M, int H,
+                       int G, int P, int N, float scale, void* o, gdn_dtype o_dtype, float* hT,
+                       void* workspace, size_t ws_bytes, void* stream) {
+    if (B < 0 || T < 0 || n_seq < 0) return GDN_ERR_INVALID_ARG;
+    if (o_dtype != GDN_F32 && o_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (B != 1 || n_seq < 1) return GDN_ERR_INVALID_ARG;
+    } else {
+        n_seq = B;
+    }
+    const int64_t rows = cu_seqlens ? T : (int64_t)B * T;
+    if (rows > 0x7fffffff || rows * (int64_t)(M > 0 ? M : 1) >= ((int64_t)1 << 31))
+        return GDN_ERR_UNSUPPORTED;
+    gdn_status s = decode_args_ok(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, (int)rows, M, H,
+                                  G, P, N);
+    if (s != GDN_OK) return s;
+    if (n_seq == 0) return GDN_OK;
+    if (rows > 0 && !o) return GDN_ERR_INVALID_ARG;
+    for (const void* p : {(const void*)h0, (const void*)o, (const void*)hT})
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const PrefillLayout L = prefill_layout(n_seq, rows, M, H, P, N, o_dtype, cu_seqlens != nullptr);
+    if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* beta = reinterpret_cast<float*>(ws + L.beta);
+    float* g = reinterpret_cast<float*>(ws + L.g);
+    if (rows > 0) {
+        s = gdp_decode_prepare(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, (int)rows, M, H, G,
+                               P, N, ws + L.q, ws + L.k, ws + L.v, beta, g, stream);
+        if (s != GDN_OK) return s;
+    }
+    const int32_t* cu_m = nullptr;
+    if (cu_seqlens) {
+        int32_t* c = reinterpret_cast<int32_t*>(ws + L.cu);
+        gdn::gdp_scale_offsets_kernel<<<(n_seq + 256) / 256, 256, 0, st>>>(cu_seqlens, n_seq, M, c);
+        s = launch_check();
+        if (s != GDN_OK) return s;
+        cu_m = c;
+    }
+    s = gdn_chunk_fwd(ws + L.q, ws + L.k, ws + L.v, GDN_BF16, g, beta, h0, cu_m, n_seq, B, T * M,
+                      H, N, P, scale, ws + L.o_all, o_dtype, hT,
+                      cu_seqlens ? ws + L.chunk : nullptr, L.total - L.chunk, 0u, stream);
+    if (s != GDN_OK || rows == 0) return s;
+    const int64_t row_units = (int64_t)H * P * (o_dtype == GDN_BF16 ? 2 : 4) / 16;
+    const int64_t want = (rows * row_units + 255) / 256;
+    const int blocks = (int)(want < (int64_t)num_sms() * 16 ? want : (int64_t)num_sms() * 16);
+    gdn::gdp_last_copy_kernel<<<blocks, 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(ws + L.o_all), rows, M, row_units, static_cast<uint4*>(o));
+    return launch_check();
+}
+
 gdn_status gdn_conv1d_fwd(const void* x, int dtype, const float* w, const float* bias, int W,
                           const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int C,
                           const void* init_state, void* final_state, int activation, void* y,

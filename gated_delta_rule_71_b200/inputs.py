@@ -160,6 +160,38 @@ def decode_inputs(w: DecodeWorkload, seed: Optional[int] = None):
     return dict(x=x, ba=ba, A_log=A_log, dt_bias=dt_bias, state=state)
 
 
+@dataclass(frozen=True)
+class PrefillWorkload:
+    name: str
+    B: int
+    T: int
+    M: int
+    H: int
+    G: int
+    P: int
+    N: int
+    seed: int = 0
+
+
+# The decode step's head configuration over a 4096-token prompt.
+GDP_PREFILL = PrefillWorkload("GDP prefill B1 T4096 M2 H32 G16 P=N=128", 1, 4096, 2, 32, 16,
+                              128, 128, seed=1005)
+
+
+def prefill_inputs(w: PrefillWorkload, seed: Optional[int] = None):
+    """x [B,T,M*H*P+M*G*N+G*N] and ba [B,T,M*H+H] bf16 rows in the decode layout,
+    A_log, dt_bias [H] fp32 (CPU tensors).  x ~ N(0,1) with the key and query
+    parts scaled by N^-1/2 (unit expected norm: the prefill uses them as given),
+    ba ~ N(0,1); gate parameters as for the chunk workloads."""
+    gen = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    M, H, G, P, N = w.M, w.H, w.G, w.P, w.N
+    x = _normal(gen, (w.B, w.T, M * H * P + M * G * N + G * N))
+    x[..., M * H * P:] *= 1.0 / math.sqrt(N)
+    ba = _normal(gen, (w.B, w.T, M * H + H))
+    A_log, dt_bias = _gate_params(gen, H)
+    return dict(x=x.to(torch.bfloat16), ba=ba.to(torch.bfloat16), A_log=A_log, dt_bias=dt_bias)
+
+
 def conv_inputs(w: ConvWorkload, seed: Optional[int] = None, lengths=None):
     """x [B, T, C] (or [1, T, C] packed, with cu_seqlens), w [C, W], bias [C], and
     init_state [n_seq, C, W-1] when the workload has one.  CPU tensors."""

@@ -197,6 +197,37 @@ gdn_status gdp_decode_step_indexed(const void* x, int64_t x_n_stride, const void
                                    int qk_l2norm, void* stream);
 
 /*
+ * gdp_prefill -- the Gated Delta Product over a whole prompt: every token row
+ * carries the decode layout (x row [value: M*H*P | key: M*G*N | query: G*N],
+ * ba row [b: M*H | a: H], as in gdp_decode_prepare), and the rule runs over the
+ * M Householder copies of each token in order -- copy m of token t is step
+ * t*M + m of a T*M-step sequence, with the query on copy M-1 and the decay on
+ * copy 0 (Megatron-Core "core.ssm.ops.gdp.decode_prepare": module description
+ * and the gdp_decode_prepare entry, whose outputs are the layouts the
+ * recurrent kernel expects for an M-length sequence per request).  o is taken
+ * at each token's last copy.  The result equals T successive gdp_decode_step
+ * calls with qk_l2norm = 0 (q and k are used as given), computed with the
+ * chunked kernels of gdn_chunk_fwd.
+ *   x, ba     : bf16 rows, B*T of them (dense) or T_total (cu_seqlens != NULL,
+ *               B == 1), row strides x_n_stride / ba_n_stride elements.
+ *   h0        : fp32 [n_seq, H, N, P] or NULL (zero).
+ *   cu_seqlens: int32 [n_seq+1] token offsets (device) or NULL.
+ *   o         : [rows, H, P] of o_dtype;  hT : fp32 [n_seq, H, N, P] or NULL.
+ *   workspace : >= gdp_prefill_workspace_size(n_seq, rows, M, H, P, N, o_dtype,
+ *               cu_seqlens != NULL) bytes, 16-byte aligned (it holds the
+ *               interleaved q/k/v/gates and the output of every copy).
+ * Errors: as gdp_decode_prepare and gdn_chunk_fwd; UNSUPPORTED when rows * M
+ * reaches 2^31.
+ */
+size_t gdp_prefill_workspace_size(int n_seq, int64_t rows, int M, int H, int P, int N,
+                                  gdn_dtype o_dtype, int packed);
+gdn_status gdp_prefill(const void* x, int64_t x_n_stride, const void* ba, int64_t ba_n_stride,
+                       const float* A_log, const float* dt_bias, const float* h0,
+                       const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int M, int H,
+                       int G, int P, int N, float scale, void* o, gdn_dtype o_dtype, float* hT,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate
  * device memory.  The sources describe no such entry point; it exists because
  * some callers have no way to provide the packed-batch workspace: code running

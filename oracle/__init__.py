@@ -220,6 +220,30 @@ def gdp_decode_step_indexed(x, ba, A_log, dt_bias, state_pool, state_idx, M, H, 
     return o, pool
 
 
+def gdp_prefill(x, ba, A_log, dt_bias, M, H, G, P, N, h0=None, cu_seqlens=None, scale=1.0):
+    """Gated Delta Product over a prompt (Megatron-Core
+    "core.ssm.ops.gdp.decode_prepare": the prepare outputs are an M-length
+    sequence per token for the recurrent rule).  x [B, T, row] / ba [B, T, row]
+    bf16 rows in the decode layout; the rule runs over the copy-interleaved
+    sequence (copy m of token t is step t*M + m) built by gdp_decode_prepare,
+    and o is read at each token's last copy.  Returns (o [B, T, H, P] fp64,
+    hT [n_seq, H, N, P] fp64)."""
+    B, T = x.shape[0], x.shape[1]
+    R = B * T
+    q, k, v, beta, g = gdp_decode_prepare(x.reshape(R, 1, -1), ba.reshape(R, 1, -1), A_log,
+                                          dt_bias, M, H, G, P, N)
+    wid = lambda u: (u.astype(np.uint32) << 16).view(np.float32)
+    q, k, v = wid(q), wid(k), wid(v)
+    seq = lambda a, d: a.reshape(B, T * M, H, d)
+    cu = None
+    if cu_seqlens is not None:
+        cu_np = cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else np.asarray(cu_seqlens)
+        cu = (cu_np.astype(np.int64) * M).astype(np.int32)
+    o, hT = gdn_fwd(seq(q, N), seq(k, N), seq(v, P), g.reshape(B, T * M, H),
+                    beta.reshape(B, T * M, H), h0=h0, cu_seqlens=cu, scale=scale)
+    return o[:, M - 1::M], hT
+
+
 def conv1d_fwd(x, w, bias=None, cu_seqlens=None, init_state=None, activation=False):
     """Causal depthwise conv1d in fp64.
 

@@ -104,6 +104,32 @@ def test_decode_rejects_bad_arguments():
     assert ix(*big, p, p, 8, p, 1.0, 1, None) == UNSUPPORTED              # M > 8
 
 
+def test_prefill_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    M, H, G, P, N, T = 2, 4, 2, 128, 128, 10
+    row = M * H * P + M * G * N + G * N
+    need = lib.gdp_prefill_workspace_size(2, 2 * T, M, H, P, N, 0, 0)
+    assert need > 2 * T * M * H * (2 * N + P) * 2  # interleaved q, k, v at least
+    assert lib.gdp_prefill_workspace_size(2, 2 * T, 0, H, P, N, 0, 0) == 0
+    big = 1 << 40
+
+    def call(**kw):
+        a = dict(x=p, xs=row, ba=p, bas=M * H + H, cu=None, n_seq=0, B=2, T=T, M=M, H=H, G=G,
+                 ws=p, wsb=big)
+        a.update(kw)
+        return lib.gdp_prefill(a["x"], a["xs"], a["ba"], a["bas"], p, p, None, a["cu"],
+                               a["n_seq"], a["B"], a["T"], a["M"], a["H"], a["G"], P, N, 1.0, p,
+                               0, p, a["ws"], a["wsb"], None)
+    assert call(G=3) == INVALID                       # H % G
+    assert call(xs=row - 1) == INVALID                # row stride shorter than a row
+    assert call(cu=p, n_seq=2, B=2) == INVALID        # packed needs B == 1
+    assert call(ws=None) == INVALID
+    assert call(wsb=need - 1) == INVALID
+    assert call(T=1 << 30) == UNSUPPORTED             # rows * M reaches 2^31
+    assert call(B=0) == 0                             # nothing to do
+
+
 def test_selftest_rejects_zero_polls():
     assert _lib.load().gdn_selftest_wait_timeout(0, None) == INVALID
 

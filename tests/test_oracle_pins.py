@@ -320,3 +320,41 @@ def test_decode_indexed_padding_and_slots():
         np.testing.assert_array_equal(new[sl], s1[0])
     for sl in (1, 3, 4):  # slots no request names are untouched
         np.testing.assert_array_equal(new[sl], pool[sl].double().numpy())
+
+
+def test_prefill_equals_successive_decode_steps():
+    # the Gated Delta Product prefill over T tokens is T decode steps in a row
+    # (q and k as given), each token's output taken at its last copy
+    B, T, M, H, G, P, N = 2, 5, 3, 4, 2, 8, 8
+    gen = torch.Generator().manual_seed(23)
+    x = torch.randn(B, T, M * H * P + M * G * N + G * N, generator=gen).to(torch.bfloat16)
+    ba = torch.randn(B, T, M * H + H, generator=gen).to(torch.bfloat16)
+    A_log = torch.rand(H, generator=gen)
+    dt_bias = torch.randn(H, generator=gen)
+    h0 = torch.randn(B, H, N, P, generator=gen) * 0.1
+    o, hT = oracle.gdp_prefill(x, ba, A_log, dt_bias, M, H, G, P, N, h0=h0, scale=0.7)
+    for b in range(B):
+        st = h0[b][None].double().numpy()
+        for t in range(T):
+            od, st = oracle.gdp_decode_step(x[b, t][None, None], ba[b, t][None, None], A_log,
+                                            dt_bias, st.astype(np.float32), M, H, G, P, N,
+                                            scale=0.7, qk_l2norm=False)
+            # the decode oracle restarts from an fp32 copy of the state each step
+            np.testing.assert_allclose(o[b, t], od[0], rtol=1e-6, atol=1e-6)
+        np.testing.assert_allclose(hT[b], st[0], rtol=1e-6, atol=1e-6)
+
+
+def test_prefill_packed_matches_dense_runs():
+    T1, T2, M, H, G, P, N = 3, 4, 2, 2, 1, 8, 8
+    gen = torch.Generator().manual_seed(29)
+    x = torch.randn(1, T1 + T2, M * H * P + M * G * N + G * N, generator=gen).to(torch.bfloat16)
+    ba = torch.randn(1, T1 + T2, M * H + H, generator=gen).to(torch.bfloat16)
+    A_log = torch.rand(H, generator=gen)
+    dt_bias = torch.randn(H, generator=gen)
+    cu = np.array([0, T1, T1 + T2], np.int32)
+    o, hT = oracle.gdp_prefill(x, ba, A_log, dt_bias, M, H, G, P, N, cu_seqlens=cu)
+    o1, h1 = oracle.gdp_prefill(x[:, :T1], ba[:, :T1], A_log, dt_bias, M, H, G, P, N)
+    o2, h2 = oracle.gdp_prefill(x[:, T1:], ba[:, T1:], A_log, dt_bias, M, H, G, P, N)
+    np.testing.assert_array_equal(o[:, :T1], o1)
+    np.testing.assert_array_equal(o[:, T1:], o2)
+    np.testing.assert_array_equal(hT, np.concatenate([h1, h2]))
