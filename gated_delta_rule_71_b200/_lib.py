@@ -32,6 +32,8 @@ SIGNATURES = {
     "gdp_prefill_workspace_size": (SZ, [I32, I64, I32, I32, I32, I32, I32, I32]),
     "gdp_prefill": (I32, [P, I64, P, I64, P, P, P, P, I32, I32, I64, I32, I32, I32, I32, I32,
                           F32, P, I32, P, P, SZ, P]),
+    "gdn_state_combine": (I32, [P, P, P, P, I64, I32, I32, P]),
+    "gdn_accumulate_f32": (I32, [P, P, I64, P]),
     "gdn_chunk_fwd_noalloc": (I32, [P, P, P, I32, P, P, P, P, I32, I32, I64, I32, I32, I32, F32,
                                     P, I32, P, U32, P]),
     "gdn_conv1d_fwd": (I32, [P, I32, P, P, I32, P, I32, I32, I64, I32, P, P, I32, P, P]),

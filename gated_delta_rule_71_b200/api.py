@@ -230,6 +230,35 @@ def gdp_prefill(x, ba, A_log, dt_bias, M, H, G, P, N, h0=None, cu_seqlens=None, 
     return o, hT
 
 
+def state_combine(A: torch.Tensor, X: torch.Tensor, C: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out = A X (+ C) for A fp32 [n,K,K], X and C fp32 [n,K,V] (gdn_state_combine)."""
+    dev = A.device
+    for t, name in ((A, "A"), (X, "X")):
+        _need(t, name, torch.float32, dev)
+    n, K, _ = A.shape
+    V = X.shape[-1]
+    if tuple(A.shape) != (n, K, K) or tuple(X.shape) != (n, K, V):
+        raise ValueError("A must be [n, K, K] and X [n, K, V]")
+    if C is not None:
+        _need(C, "C", torch.float32, dev)
+        if tuple(C.shape) != (n, K, V):
+            raise ValueError("C must be [n, K, V]")
+    if out is None:
+        out = torch.empty((n, K, V), dtype=torch.float32, device=dev)
+    _lib.call("gdn_state_combine", _ptr(A), _ptr(X), _ptr(C), _ptr(out), n, K, V, _stream(A))
+    return out
+
+
+def accumulate_f32(y: torch.Tensor, x: torch.Tensor) -> None:
+    """y += x for fp32 tensors of the same size (gdn_accumulate_f32)."""
+    _need(y, "y", torch.float32, y.device)
+    _need(x, "x", torch.float32, y.device)
+    if y.numel() != x.numel():
+        raise ValueError("y and x must have the same number of elements")
+    _lib.call("gdn_accumulate_f32", _ptr(y), _ptr(x), y.numel(), _stream(y))
+
+
 def device_status(device=None) -> int:
     """Reads and clears the device status word (synchronises the current stream)."""
     s = torch.cuda.current_stream(device).cuda_stream

@@ -269,3 +269,56 @@ __global__ void __launch_bounds__(256) gdp_last_copy_kernel(const uint4* __restr
 }
 
 }  // namespace gdn
+
+namespace gdn {
+
+// ------------------------------------------------------- context parallelism
+// out[i] = A[i] X[i] + C[i] for a batch of (K x K) . (K x V) fp32 products: the
+// state entering a sequence segment from the previous segment's transition
+// matrix, incoming state and local final state.  One block per (matrix, 32
+// output columns); the K x 32 slab of X and 32-row panels of A go through
+// shared memory.  Small next to the chunked passes it joins.
+template <int K>
+__global__ void __launch_bounds__(256) state_combine_kernel(const float* __restrict__ A,
+                                                            const float* __restrict__ X,
+                                                            const float* __restrict__ Cm,
+                                                            float* __restrict__ out, int V) {
+    __shared__ float xs[K][33];
+    __shared__ float as[32][K + 1];
+    const int i = blockIdx.y, c0 = 32 * blockIdx.x;
+    const int64_t aoff = (int64_t)i * K * K, xoff = (int64_t)i * K * V;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 row groups
+    for (int e = threadIdx.x; e < K * 32; e += 256) {
+        const int r = e >> 5, c = e & 31;
+        xs[r][c] = (c0 + c < V) ? X[xoff + (int64_t)r * V + c0 + c] : 0.f;
+    }
+    for (int rp = 0; rp < K; rp += 32) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < 32 * K; e += 256) {
+            const int r = e / K, kk = e - r * K;
+            as[r][kk] = A[aoff + (int64_t)(rp + r) * K + kk];
+        }
+        __syncthreads();
+        for (int r = ty; r < 32; r += 8) {
+            float acc = 0.f;
+#pragma unroll 8
+            for (int kk = 0; kk < K; ++kk) acc = fmaf(as[r][kk], xs[kk][tx], acc);
+            const int row = rp + r, col = c0 + tx;
+            if (col < V) {
+                const int64_t o = xoff + (int64_t)row * V + col;
+                out[o] = acc + (Cm ? Cm[o] : 0.f);
+            }
+        }
+    }
+}
+
+// y[i] += x[i] (fp32), grid-stride.
+__global__ void __launch_bounds__(256) accumulate_f32_kernel(float* __restrict__ y,
+                                                             const float* __restrict__ x,
+                                                             int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        y[i] += x[i];
+}
+
+}  // namespace gdn

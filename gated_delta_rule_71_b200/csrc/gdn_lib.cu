@@ -409,6 +409,31 @@ gdn_status gdp_prefill(const void* x, int64_t x_n_stride, const void* ba, int64_
     return launch_check();
 }
 
+gdn_status gdn_state_combine(const float* A, const float* X, const float* C, float* out,
+                             int64_t count, int K, int V, void* stream) {
+    if (count < 0 || !head_dim_ok(K) || V < 1) return count < 0 ? GDN_ERR_INVALID_ARG
+                                                                 : GDN_ERR_UNSUPPORTED;
+    if (count == 0) return GDN_OK;
+    if (!A || !X || !out || out == X) return GDN_ERR_INVALID_ARG;
+    if (count > 65535) return GDN_ERR_UNSUPPORTED;
+    dim3 grid((V + 31) / 32, (unsigned)count);
+    cudaStream_t st = as_stream(stream);
+    if (K == 128) gdn::state_combine_kernel<128><<<grid, 256, 0, st>>>(A, X, C, out, V);
+    else if (K == 64) gdn::state_combine_kernel<64><<<grid, 256, 0, st>>>(A, X, C, out, V);
+    else gdn::state_combine_kernel<32><<<grid, 256, 0, st>>>(A, X, C, out, V);
+    return launch_check();
+}
+
+gdn_status gdn_accumulate_f32(float* y, const float* x, int64_t n, void* stream) {
+    if (n < 0) return GDN_ERR_INVALID_ARG;
+    if (n == 0) return GDN_OK;
+    if (!y || !x) return GDN_ERR_INVALID_ARG;
+    const int64_t want = (n + 255) / 256;
+    const int blocks = (int)(want < (int64_t)num_sms() * 16 ? want : (int64_t)num_sms() * 16);
+    gdn::accumulate_f32_kernel<<<blocks, 256, 0, as_stream(stream)>>>(y, x, n);
+    return launch_check();
+}
+
 gdn_status gdn_conv1d_fwd(const void* x, int dtype, const float* w, const float* bias, int W,
                           const int32_t* cu_seqlens, int n_seq, int B, int64_t T, int C,
                           const void* init_state, void* final_state, int activation, void* y,

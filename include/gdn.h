@@ -308,6 +308,26 @@ gdn_status gdn_conv1d_update(const void* x, int dtype, const float* w, const flo
                              int activation, void* y, void* stream);
 
 /*
+ * Context parallelism over T.  The rule is linear in (h0, v) jointly, so a
+ * sequence split into segments runs as: each segment from a zero state
+ * (o_loc, h_loc); its transition matrix M (h_T of the segment with v = 0 and
+ * h0 = I, key x key); the state entering segment r is s_{r-1}, where
+ * s_0 = h_loc_0 and s_j = M_j s_{j-1} + h_loc_j; and segment r's output is
+ * o_loc plus the output of a v = 0 pass from s_{r-1}.  These two calls are
+ * the pieces of that which are not gdn_chunk_fwd itself.  (ZzCompute's "Chunk
+ * Forward H" carries the state across chunks; this carries it across
+ * segments the same way.)
+ *
+ * gdn_state_combine -- out[i] = A[i] X[i] (+ C[i]) for `count` matrices:
+ *   A fp32 [count, K, K]; X, C, out fp32 [count, K, V]; C may be NULL; out may
+ *   equal C but not X.  K in {32, 64, 128}; count <= 65535.
+ * gdn_accumulate_f32 -- y[i] += x[i] for n fp32 elements.
+ */
+gdn_status gdn_state_combine(const float* A, const float* X, const float* C, float* out,
+                             int64_t count, int K, int V, void* stream);
+gdn_status gdn_accumulate_f32(float* y, const float* x, int64_t n, void* stream);
+
+/*
  * gdn_device_status -- reads and clears the device status word on the current
  * device.  Kernels that wait on the device (mbarrier waits in the tensor-core
  * kernel) give up after a bounded number of polls, record GDN_ERR_TIMEOUT

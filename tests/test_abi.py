@@ -130,6 +130,21 @@ def test_prefill_rejects_bad_arguments():
     assert call(B=0) == 0                             # nothing to do
 
 
+def test_cp_helpers_reject_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(256)
+    q = ctypes.c_void_p(512)
+    assert lib.gdn_state_combine(p, p, None, q, 4, 96, 128, None) == UNSUPPORTED  # K
+    assert lib.gdn_state_combine(p, p, None, q, -1, 128, 128, None) == INVALID
+    assert lib.gdn_state_combine(p, p, None, q, 1 << 17, 128, 128, None) == UNSUPPORTED
+    assert lib.gdn_state_combine(None, p, None, q, 4, 128, 128, None) == INVALID
+    assert lib.gdn_state_combine(p, p, None, p, 4, 128, 128, None) == INVALID  # out == X
+    assert lib.gdn_state_combine(p, p, None, q, 0, 128, 128, None) == 0
+    assert lib.gdn_accumulate_f32(p, None, 10, None) == INVALID
+    assert lib.gdn_accumulate_f32(p, p, -1, None) == INVALID
+    assert lib.gdn_accumulate_f32(p, p, 0, None) == 0
+
+
 def test_selftest_rejects_zero_polls():
     assert _lib.load().gdn_selftest_wait_timeout(0, None) == INVALID
 
