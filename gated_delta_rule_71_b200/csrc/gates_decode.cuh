@@ -82,31 +82,36 @@ __global__ void __launch_bounds__(256) gdp_prepare_kernel(
 // (Megatron-Core "core.ssm.ops.gdp.decode_prepare", module description: the
 // batch is padded upstream with -1 slots).  A slot >= n_slots is handled the
 // same way and records GDN_ERR_INVALID_ARG in the device status word.  The
-// fp32 state [N, P] lives in registers: warp w owns key rows [w*N/8, (w+1)*N/8), lane l owns value
-// columns [l*P/32, (l+1)*P/32), so every row is read and written as one
-// coalesced 512-byte (P = 128) warp access.  Column reductions over the key
+// value columns of the state never interact, so a (request, head) is split
+// over P / PB blocks of PB columns each (smaller blocks: more of them resident
+// per SM to overlap one block's loads with another's arithmetic).  The block's
+// fp32 state slab [N, PB] lives in registers: warp w owns key rows
+// [w*N/8, (w+1)*N/8), lane l owns columns [l*PB/32, (l+1)*PB/32), so every row
+// is read and written as one coalesced warp access.  Column reductions over the key
 // axis go through shared memory.  The state is read once and written once:
 // the kernel is HBM-bound on 2*N*P*4 bytes per (request, head).
 constexpr int kDecWarps = 8;
 constexpr int kDecMaxM = 8;
 
-template <int N, int P>
-__global__ void __launch_bounds__(256) gdp_step_kernel(
+template <int N, int P, int PB>
+__global__ void __launch_bounds__(256, (PB <= 64 ? 4 : 2)) gdp_step_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t xs, const __nv_bfloat16* __restrict__ ba,
     int64_t bas, const float* __restrict__ A_log, const float* __restrict__ dt_bias, int M, int H,
     int G, float* __restrict__ state, const int32_t* __restrict__ state_idx, int n_slots,
     __nv_bfloat16* __restrict__ o, float scale, int l2) {
     constexpr int RPW = N / kDecWarps;  // rows per warp
-    constexpr int CPL = P / 32;         // columns per lane
+    constexpr int CPL = PB / 32;        // columns per lane
+    constexpr int NPART = P / PB;
     __shared__ float kv[kDecMaxM][N];
-    __shared__ float vv[kDecMaxM][P];
+    __shared__ float vv[kDecMaxM][PB];
     __shared__ float qv[N];
-    __shared__ float red[kDecWarps][P];
-    __shared__ float uu[P];
+    __shared__ float red[kDecWarps][PB];
+    __shared__ float uu[PB];
     __shared__ float gate_b[kDecMaxM];
     __shared__ float gate_e;
 
-    const int rh = blockIdx.x;  // request * H + head
+    const int rh = blockIdx.x / NPART;  // request * H + head
+    const int p0 = (blockIdx.x - rh * NPART) * PB;  // first value column of this block
     const int r = rh / H, h = rh - r * H;
     const int hpg = H / G, grp = h / hpg;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -116,12 +121,12 @@ __global__ void __launch_bounds__(256) gdp_step_kernel(
     const int slot = state_idx ? state_idx[r] : r;
     if (slot < 0 || slot >= n_slots) {  // padding (uniform across the block)
         if (slot >= n_slots && threadIdx.x == 0) record_status(GDN_ERR_INVALID_ARG);
-        if (threadIdx.x < P) o[(int64_t)rh * P + threadIdx.x] = __float2bfloat16_rn(0.f);
+        if (threadIdx.x < PB) o[(int64_t)rh * P + p0 + threadIdx.x] = __float2bfloat16_rn(0.f);
         return;
     }
 
     // 1. issue the state loads first (the only large traffic)
-    float* st = state + ((int64_t)slot * H + h) * N * P;
+    float* st = state + ((int64_t)slot * H + h) * N * P + p0;
     float s[RPW][CPL];
 #pragma unroll
     for (int rr = 0; rr < RPW; ++rr) {
@@ -155,9 +160,9 @@ __global__ void __launch_bounds__(256) gdp_step_kernel(
 #pragma unroll
         for (int i = 0; i < N / 32; ++i) dst[lane + 32 * i] = e[i] * inv;
     }
-    for (int i = threadIdx.x; i < M * P; i += blockDim.x) {
-        const int m = i / P, j = i - m * P;
-        vv[m][j] = __bfloat162float(xr[((int64_t)m * H + h) * P + j]);
+    for (int i = threadIdx.x; i < M * PB; i += blockDim.x) {
+        const int m = i / PB, j = i - m * PB;
+        vv[m][j] = __bfloat162float(xr[((int64_t)m * H + h) * P + p0 + j]);
     }
     if (threadIdx.x < M) gate_b[threadIdx.x] = write_gate(__bfloat162float(br[threadIdx.x * H + h]));
     if (threadIdx.x == M)
@@ -174,19 +179,19 @@ __global__ void __launch_bounds__(256) gdp_step_kernel(
 #pragma unroll
                 for (int c = 0; c < CPL; ++c) s[rr][c] *= e0;
         }
-        float p[CPL];
+        float pp[CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) p[c] = 0.f;
+        for (int c = 0; c < CPL; ++c) pp[c] = 0.f;
 #pragma unroll
         for (int rr = 0; rr < RPW; ++rr) {
             const float kk = kv[m][warp * RPW + rr];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) p[c] = fmaf(s[rr][c], kk, p[c]);
+            for (int c = 0; c < CPL; ++c) pp[c] = fmaf(s[rr][c], kk, pp[c]);
         }
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = p[c];
+        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = pp[c];
         __syncthreads();
-        if (threadIdx.x < P) {
+        if (threadIdx.x < PB) {
             float d = 0.f;
 #pragma unroll
             for (int w = 0; w < kDecWarps; ++w) d += red[w][threadIdx.x];
@@ -204,29 +209,7 @@ __global__ void __launch_bounds__(256) gdp_step_kernel(
         }
     }
 
-    // 4. output at the last copy: o = scale * S^T q
-    {
-        float p[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) p[c] = 0.f;
-#pragma unroll
-        for (int rr = 0; rr < RPW; ++rr) {
-            const float qq = qv[warp * RPW + rr];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) p[c] = fmaf(s[rr][c], qq, p[c]);
-        }
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = p[c];
-        __syncthreads();
-        if (threadIdx.x < P) {
-            float d = 0.f;
-#pragma unroll
-            for (int w = 0; w < kDecWarps; ++w) d += red[w][threadIdx.x];
-            o[(int64_t)rh * P + threadIdx.x] = __float2bfloat16_rn(scale * d);
-        }
-    }
-
-    // 5. write the state back in place
+    // 4. write the state back in place, then the output at the last copy
 #pragma unroll
     for (int rr = 0; rr < RPW; ++rr) {
         float* dst = st + (int64_t)(warp * RPW + rr) * P + lane * CPL;
@@ -236,6 +219,26 @@ __global__ void __launch_bounds__(256) gdp_step_kernel(
             *reinterpret_cast<float2*>(dst) = make_float2(s[rr][0], s[rr][1]);
         } else {
             dst[0] = s[rr][0];
+        }
+    }
+    {
+        float pp[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) pp[c] = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < RPW; ++rr) {
+            const float qq = qv[warp * RPW + rr];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) pp[c] = fmaf(s[rr][c], qq, pp[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = pp[c];
+        __syncthreads();
+        if (threadIdx.x < PB) {
+            float d = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) d += red[w][threadIdx.x];
+            o[(int64_t)rh * P + p0 + threadIdx.x] = __float2bfloat16_rn(scale * d);
         }
     }
 }

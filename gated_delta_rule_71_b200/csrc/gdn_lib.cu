@@ -287,16 +287,20 @@ gdn_status gdp_decode_step_indexed(const void* x, int64_t x_n_stride, const void
     if (n_slots > 0 && (!state || !aligned16(state))) return GDN_ERR_INVALID_ARG;
     if (state_idx && (reinterpret_cast<uintptr_t>(state_idx) & 3u)) return GDN_ERR_INVALID_ARG;
     if (M > gdn::kDecMaxM) return GDN_ERR_UNSUPPORTED;
-    if ((int64_t)n * H > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)n * H * 2 > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
     using bf = __nv_bfloat16;
     const int nb = n * H;
     cudaStream_t st = as_stream(stream);
+    // 64-column slabs for P >= 64 (two blocks per (request, head) at P = 128): four
+    // blocks fit per SM, so one block's state loads overlap another's arithmetic
+    // (measured 0.787 -> 0.822 of the HBM copy bandwidth at n=256 M=2 H=32 G=16 P=N=128;
+    // 32-column slabs were slower, 0.695)
 #define GDN_DEC(NN, PP)                                                                          \
     if (N == NN && P == PP) {                                                                    \
-        gdn::gdp_step_kernel<NN, PP><<<nb, 256, 0, st>>>((const bf*)x, x_n_stride, (const bf*)ba, \
-                                                          ba_n_stride, A_log, dt_bias, M, H, G,  \
-                                                          state, state_idx, n_slots, (bf*)o,     \
-                                                          scale, qk_l2norm);                     \
+        constexpr int PB = PP >= 64 ? 64 : PP;                                                   \
+        gdn::gdp_step_kernel<NN, PP, PB><<<nb * (PP / PB), 256, 0, st>>>(                         \
+            (const bf*)x, x_n_stride, (const bf*)ba, ba_n_stride, A_log, dt_bias, M, H, G, state, \
+            state_idx, n_slots, (bf*)o, scale, qk_l2norm);                                       \
         return launch_check();                                                                   \
     }
     GDN_DEC(128, 128) GDN_DEC(128, 64) GDN_DEC(128, 32)
