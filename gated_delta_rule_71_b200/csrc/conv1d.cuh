@@ -22,6 +22,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdn {
 
@@ -71,9 +72,33 @@ __device__ __forceinline__ void conv_store(T* p, const float (&v)[NV]) {
     }
 }
 
-// SiLU with the fast exponential and divide (bf16 outputs carry 8 bits; the
-// fp32 error of __expf / __fdividef stays below 2^-20 relative here).
-__device__ __forceinline__ float conv_silu(float y) { return __fdividef(y, 1.0f + __expf(-y)); }
+// SiLU as y / (1 + 2^(-y log2 e)) from the hardware's approximate base-2
+// exponential and reciprocal (ex2.approx.ftz / rcp.approx.ftz, each within a
+// few fp32 ulp).  Rounding -y log2 e perturbs the exponential by at most
+// |y| 2^-24 relative, so for |y| < 64 the result is within 2^-17 of SiLU
+// relative, far inside the 8 bits of a bf16 output; below y = -87 the
+// reciprocal flushes to zero and so does the result (|SiLU| < 2^-119 there).
+// The packed form does the same per lane (each f32x2 lane one IEEE op), so
+// every conv kernel gives the same bits.
+__device__ __forceinline__ float conv_ex2(float t) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(t));
+    return r;
+}
+__device__ __forceinline__ float conv_rcp(float d) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+    return r;
+}
+constexpr float kNegLog2e = -1.4426950408889634f;
+__device__ __forceinline__ float conv_silu(float y) {
+    return y * conv_rcp(1.0f + conv_ex2(y * kNegLog2e));
+}
+__device__ __forceinline__ float2 conv_silu2(float2 y) {
+    const float2 t = __fmul2_rn(y, make_float2(kNegLog2e, kNegLog2e));
+    const float2 d = __fadd2_rn(make_float2(1.f, 1.f), make_float2(conv_ex2(t.x), conv_ex2(t.y)));
+    return __fmul2_rn(y, make_float2(conv_rcp(d.x), conv_rcp(d.y)));
+}
 
 // One row's NV channels as loaded (16-byte unit, or NV scalars), converted later.
 template <typename T, int NV, bool V16 = (NV * sizeof(T) == 16)>
@@ -312,6 +337,188 @@ __global__ void __launch_bounds__(128) conv1d_update_kernel(const ConvUpdateArgs
             }
         }
         conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
+    }
+}
+
+}  // namespace gdn
+
+// ------------------------------------------------ conv1d forward, TMA stream
+// The same computation for bf16, W = 4 and C a multiple of 256, restructured
+// so the bytes in flight do not live in registers: a CTA owns a strip of 256
+// channels and one contiguous range of rows.  A producer warp streams 32-row x
+// 256-channel tiles (16 KB) into a three-stage ring with TMA; four compute
+// warps (two channels per thread, so a thread owns one 4-byte column of the
+// tile) take a tile's 32 rows into registers and write the 32 outputs back
+// over them in place; the producer then stores the tile with TMA and, once
+// the store has read it, loads the stage's next tile.
+// Inside one sequence the 32 rows of a tile are independent given their
+// inputs, so that path is unrolled without branches; a tile that holds a
+// sequence boundary or the end of the range takes the row-by-row path.
+namespace gdn {
+namespace cvt {
+constexpr int TR = 32;        // rows per tile
+constexpr int TC = 256;       // channels per strip
+constexpr int NS = 3;         // ring stages (four CTAs fit on an SM)
+constexpr int kThreads = 160; // 4 compute warps + the producer warp
+constexpr uint32_t TILE = TR * TC * 2;
+constexpr uint32_t OFF_BAR = NS * TILE;
+constexpr uint32_t SMEM = OFF_BAR + 2 * NS * 8 + 128;  // + alignment slack
+constexpr uint32_t kPolls = 1u << 22;
+}  // namespace cvt
+
+struct ConvTmaParams {
+    CUtensorMap tx, ty;  // x, y [rows, C] bf16, boxes of TR rows x TC channels, no swizzle
+    ConvArgs a;
+    int64_t rows_per_cta;  // a multiple of TR
+};
+
+template <bool ACT>
+__global__ void __launch_bounds__(cvt::kThreads) conv1d_fwd_tma_kernel(
+    const __grid_constant__ ConvTmaParams p) {
+    using bf = __nv_bfloat16;
+    constexpr int H = 3;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    uint8_t* base = smem_raw + (((raw_u32 + 127u) & ~127u) - raw_u32);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + cvt::OFF_BAR);
+    uint64_t* done = full + cvt::NS;  // outputs of the stage's tile written
+    const ConvArgs& a = p.a;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cs = blockIdx.x * cvt::TC;  // first channel of the strip
+    const int64_t rbeg = (int64_t)blockIdx.y * p.rows_per_cta;
+    const int64_t rend = rbeg + p.rows_per_cta < a.rows ? rbeg + p.rows_per_cta : a.rows;
+    if (rbeg >= rend) return;
+    const int ntiles = (int)((rend - rbeg + cvt::TR - 1) / cvt::TR);
+    if (tid == 0) {
+        for (int i = 0; i < cvt::NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&done[i], 4);  // one arrive per compute warp
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == 4) {  // producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&p.tx);
+            tc::prefetch_tmap(&p.ty);
+            auto load = [&](int i) {  // tile i into stage i % NS
+                const int st_ = i % cvt::NS;
+                tc::mbar_arrive_expect_tx(&full[st_], cvt::TILE);
+                tc::tma_load_2d(base + st_ * cvt::TILE, &p.tx, cs,
+                                (int)(rbeg + (int64_t)i * cvt::TR), &full[st_]);
+            };
+            int issued = 0;
+            for (; issued < cvt::NS && issued < ntiles; ++issued) load(issued);
+            int stored = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int st_ = i % cvt::NS;
+                if (!mbar_wait(&done[st_], (i / cvt::NS) & 1, cvt::kPolls)) break;
+                tc::tma_store_2d(&p.ty, smem_u32(base + st_ * cvt::TILE), cs,
+                                 (int)(rbeg + (int64_t)i * cvt::TR));
+                tc::bulk_commit();
+                stored = i + 1;
+                if (i + cvt::NS < ntiles) {
+                    tc::bulk_wait_read0();  // the store has read the stage
+                    load(i + cvt::NS);
+                    issued = i + cvt::NS + 1;
+                }
+            }
+            tc::bulk_wait0();
+            // after a wait gave up: no load may still be landing when the CTA leaves
+            for (int i = stored; i < issued; ++i)
+                if (!mbar_wait(&full[i % cvt::NS], (i / cvt::NS) & 1, cvt::kPolls)) break;
+        }
+        return;
+    }
+    const int c0 = cs + 2 * tid;  // this thread's two channels
+    const bf* x = static_cast<const bf*>(a.x);
+    const bf* init = static_cast<const bf*>(a.init);
+    bf* fin = static_cast<bf*>(a.fin);
+    // the two channels side by side: packed fp32 pairs (each lane one IEEE fma)
+    float2 wt[4], bs;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) wt[i] = make_float2(a.w[(int64_t)c0 * 4 + i], a.w[(int64_t)(c0 + 1) * 4 + i]);
+    bs = a.bias ? make_float2(a.bias[c0], a.bias[c0 + 1]) : make_float2(0.f, 0.f);
+    int s;
+    int64_t st, en;
+    conv_find_seq(a, rbeg, s, st, en);
+    float2 win[H];
+    auto fill = [&](int64_t r) {  // the H inputs before row r
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            const int64_t pos = r - H + i;
+            float v[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (pos >= st)
+                    v[j] = __bfloat162float(x[pos * a.C + c0 + j]);
+                else if (init)
+                    v[j] = __bfloat162float(init[((int64_t)s * a.C + c0 + j) * H + (H + (pos - st))]);
+                else
+                    v[j] = 0.f;
+            }
+            win[i] = make_float2(v[0], v[1]);
+        }
+    };
+    // one row: output from the window and the row's inputs, then shift them in
+    auto row = [&](uint32_t in, uint32_t* out) {
+        __nv_bfloat162 b2;
+        memcpy(&b2, &in, 4);
+        const float2 xc = __bfloat1622float2(b2);
+        float2 acc = bs;
+#pragma unroll
+        for (int k = 0; k < H; ++k) acc = __ffma2_rn(wt[k], win[k], acc);
+        acc = __ffma2_rn(wt[H], xc, acc);
+        if (ACT) acc = conv_silu2(acc);
+        const __nv_bfloat162 ob = __floats2bfloat162_rn(acc.x, acc.y);
+        uint32_t ou;
+        memcpy(&ou, &ob, 4);
+        *out = ou;
+        win[0] = win[1];
+        win[1] = win[2];
+        win[2] = xc;
+    };
+    auto write_fin = [&]() {  // the sequence's last W-1 inputs, oldest first
+#pragma unroll
+        for (int k = 0; k < H; ++k) {
+            fin[((int64_t)s * a.C + c0) * H + k] = __float2bfloat16_rn(win[k].x);
+            fin[((int64_t)s * a.C + c0 + 1) * H + k] = __float2bfloat16_rn(win[k].y);
+        }
+    };
+    fill(rbeg);
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+        const int si = i % cvt::NS;
+        if (ok) ok = mbar_wait(&full[si], (i / cvt::NS) & 1, cvt::kPolls);
+        uint32_t* tio = reinterpret_cast<uint32_t*>(base + si * cvt::TILE) + tid;
+        const int64_t t0 = rbeg + (int64_t)i * cvt::TR;
+        if (t0 + cvt::TR <= en && t0 + cvt::TR <= rend) {
+            uint32_t in[cvt::TR];
+#pragma unroll
+            for (int rr = 0; rr < cvt::TR; ++rr) in[rr] = tio[rr * (cvt::TC / 2)];
+#pragma unroll
+            for (int rr = 0; rr < cvt::TR; ++rr) row(in[rr], tio + rr * (cvt::TC / 2));
+            if (fin && t0 + cvt::TR == en) write_fin();
+        } else {
+            for (int rr = 0; rr < cvt::TR; ++rr) {
+                const int64_t r = t0 + rr;
+                if (r >= rend) break;
+                if (r == en) {  // next (non-empty) sequence
+                    do {
+                        ++s;
+                        st = a.cu ? (int64_t)a.cu[s] : (int64_t)s * a.T;
+                        en = a.cu ? (int64_t)a.cu[s + 1] : st + a.T;
+                    } while (en <= r);
+                    fill(r);  // all W-1 taps precede the new sequence: no row loads
+                }
+                row(tio[rr * (cvt::TC / 2)], tio + rr * (cvt::TC / 2));
+                if (fin && r == en - 1) write_fin();
+            }
+        }
+        // rows past the range's end are past the tensor's end: the store clips them
+        tc::fence_async_smem();  // the outputs are visible to the TMA store
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&done[si]);
     }
 }
 

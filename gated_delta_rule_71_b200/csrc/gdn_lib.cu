@@ -92,6 +92,46 @@ gdn_status conv_fwd_w(const gdn::ConvArgs& a, int W, cudaStream_t st) {
     }
 }
 
+// The TMA-streamed variant (bf16, W = 4, C % 256 == 0, 16-byte aligned x, y):
+// strips of 256 channels x ranges of whole 32-row tiles, about one wave of
+// four CTAs per SM.  Returns GDN_ERR_UNSUPPORTED when the tensor map cannot
+// be built, so the caller can launch the register-streamed kernel instead.
+template <bool ACT>
+gdn_status launch_conv_fwd_tma(const gdn::ConvArgs& a, cudaStream_t st) {
+    using namespace gdn;
+    ConvTmaParams p;
+    memset(&p, 0, sizeof(p));
+    tcf::EncodeTiled enc = tcf::get_encode();
+    if (!enc) return GDN_ERR_UNSUPPORTED;
+    cuuint64_t dims[2] = {(cuuint64_t)a.C, (cuuint64_t)a.rows};
+    cuuint64_t strides[1] = {(cuuint64_t)a.C * 2};
+    cuuint32_t box[2] = {(cuuint32_t)cvt::TC, (cuuint32_t)cvt::TR};
+    cuuint32_t estr[2] = {1, 1};
+    CUtensorMap* maps[2] = {&p.tx, &p.ty};
+    const void* ptrs[2] = {a.x, a.y};
+    for (int i = 0; i < 2; ++i)
+        if (enc(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptrs[i]), dims,
+                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GDN_ERR_UNSUPPORTED;
+    p.a = a;
+    const int strips = a.C / cvt::TC;
+    const int64_t tiles = (a.rows + cvt::TR - 1) / cvt::TR;
+    int64_t per = (int64_t)num_sms() * 4 / strips;  // row ranges per strip
+    if (per < 1) per = 1;
+    const int64_t tiles_per_cta = (tiles + per - 1) / per;
+    p.rows_per_cta = tiles_per_cta * cvt::TR;
+    const int64_t ny = (a.rows + p.rows_per_cta - 1) / p.rows_per_cta;
+    if (ny > 65535) return GDN_ERR_UNSUPPORTED;
+    auto kern = conv1d_fwd_tma_kernel<ACT>;
+    gdn_status s = cuda_check(
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cvt::SMEM));
+    if (s != GDN_OK) return s;
+    kern<<<dim3((unsigned)strips, (unsigned)ny), cvt::kThreads, cvt::SMEM, st>>>(p);
+    return launch_check();
+}
+
 template <typename T>
 gdn_status conv_fwd_t(const gdn::ConvArgs& a, int W, bool act, bool vec, cudaStream_t st) {
     constexpr int NV = gdn::ConvVec<T>::N;
@@ -455,7 +495,16 @@ gdn_status gdn_conv1d_fwd(const void* x, int dtype, const float* w, const float*
                      (!init_state || aligned16(init_state)) && (!final_state || aligned16(final_state));
     gdn::ConvArgs a{x, w, bias, cu_seqlens, n_seq, T, rows, C, init_state, final_state, y};
     cudaStream_t st = as_stream(stream);
-    if (rows > 0) {
+    const bool tma = dtype == GDN_BF16 && W == 4 && C % gdn::cvt::TC == 0 && aligned16(x) &&
+                     aligned16(y) && rows < ((int64_t)1 << 30);
+    bool rows_done = false;
+    if (rows > 0 && tma) {
+        gdn_status s = activation == 1 ? launch_conv_fwd_tma<true>(a, st)
+                                       : launch_conv_fwd_tma<false>(a, st);
+        if (s != GDN_OK && s != GDN_ERR_UNSUPPORTED) return s;
+        if (s == GDN_OK) rows_done = true;
+    }
+    if (rows > 0 && !rows_done) {
         gdn_status s = dtype == GDN_BF16
                            ? conv_fwd_t<__nv_bfloat16>(a, W, activation == 1, vec, st)
                            : conv_fwd_t<float>(a, W, activation == 1, vec, st);

@@ -177,3 +177,48 @@ def test_decode_width_update(cuda_device):
                                    activation=True)
     _check(y, ry, torch.bfloat16, _update_term_sum(inp))
     np.testing.assert_array_equal(state.float().cpu().numpy(), rst)
+
+
+# bf16, W = 4 and C a multiple of 256 take the TMA-streamed kernel (256-channel
+# strips, 32-row tiles, contiguous row ranges per CTA); other shapes take the
+# register-streamed one.  The two evaluate the same fp32 fma sequence.
+
+@pytest.mark.parametrize("activation", [True, False])
+@pytest.mark.parametrize("init", [True, False])
+def test_tma_path_varlen_edges(cuda_device, activation, init):
+    # lengths around the 32-row tile and the W-1 halo, empty sequences, and a
+    # long tail so row ranges of several tiles start inside sequences
+    lens = [1, 2, 3, 0, 4, 31, 32, 33, 0, 63, 64, 65, 5, 127, 128, 129, 2, 9000, 3, 2900]
+    wl = I.ConvWorkload("t", 1, sum(lens), 512, 4, torch.bfloat16, n_seq_varlen=len(lens),
+                        init_state=init, seed=18)
+    y, fin, ry, rfin, S = _run_fwd(cuda_device, wl, lengths=lens, activation=activation)
+    _check(y, ry, torch.bfloat16, S)
+    np.testing.assert_array_equal(fin.float().cpu().numpy(), rfin)
+    assert gdn.device_status() == 0
+
+
+def test_tma_path_dense_ragged_tail(cuda_device):
+    # 3 x 4111 rows: a partial last tile, sequences starting inside tiles
+    wl = I.ConvWorkload("t", 3, 4111, 256, 4, torch.bfloat16, init_state=True, seed=19)
+    y, fin, ry, rfin, S = _run_fwd(cuda_device, wl)
+    _check(y, ry, torch.bfloat16, S)
+    np.testing.assert_array_equal(fin.float().cpu().numpy(), rfin)
+    assert gdn.device_status() == 0
+
+
+def test_tma_path_bit_equal_to_register_path(cuda_device):
+    # C = 768 goes through the TMA kernel, C = 776 (not a multiple of 256)
+    # through the register kernel; per channel the results must be identical.
+    lens = [700, 0, 1, 2300, 77]
+    wl = I.ConvWorkload("t", 1, sum(lens), 776, 4, torch.bfloat16, n_seq_varlen=len(lens),
+                        init_state=True, seed=20)
+    inp = I.conv_inputs(wl, lengths=lens)
+    d = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    y_r, f_r = gdn.conv1d_fwd(d["x"], d["w"], d["bias"], cu_seqlens=d["cu_seqlens"],
+                              init_state=d["init_state"], activation=True, final_state=True)
+    y_t, f_t = gdn.conv1d_fwd(d["x"][..., :768].contiguous(), d["w"][:768].contiguous(),
+                              d["bias"][:768].contiguous(), cu_seqlens=d["cu_seqlens"],
+                              init_state=d["init_state"][:, :768].contiguous(), activation=True,
+                              final_state=True)
+    assert torch.equal(y_t, y_r[..., :768])
+    assert torch.equal(f_t, f_r[:, :768])
