@@ -261,7 +261,8 @@ struct ConvUpdateArgs {
     void* y;             // [n, C]
 };
 
-constexpr int kConvReqs = 8;  // requests per thread in the update (weights loaded once)
+constexpr int kConvReqs = 16;  // requests per thread in the update (weights loaded once)
+constexpr int kConvBatchReqs = 4;  // of which loaded together ahead of their stores
 
 // Grid: x over groups of NV channels (128 threads per block), y over groups of
 // kConvReqs requests.  Requests must name distinct slots (each slot's window is
@@ -275,13 +276,98 @@ __global__ void __launch_bounds__(128) conv1d_update_kernel(const ConvUpdateArgs
     T* y = static_cast<T*>(a.y);
     T* state = static_cast<T*>(a.state);
     float wt[W][NV], bs[NV];
+    // a channel's W = 4 taps (and four channels' biases) are one 16-byte unit
+    const bool w16 = W == 4 && (reinterpret_cast<uintptr_t>(a.w) & 15u) == 0;
+    const bool b16 = NV % 4 == 0 && a.bias && (reinterpret_cast<uintptr_t>(a.bias) & 15u) == 0;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
+        if (w16) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(a.w + (int64_t)(c0 + j) * W));
+            const float t4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < W; ++i) wt[i][j] = a.w[(int64_t)(c0 + j) * W + i];
-        bs[j] = a.bias ? a.bias[c0 + j] : 0.f;
+            for (int i = 0; i < W; ++i) wt[i][j] = t4[i < 4 ? i : 0];
+        } else {
+#pragma unroll
+            for (int i = 0; i < W; ++i) wt[i][j] = a.w[(int64_t)(c0 + j) * W + i];
+        }
+        if (b16) {
+            if (j % 4 == 0) {
+                const float4 v = __ldg(reinterpret_cast<const float4*>(a.bias + c0 + j));
+                bs[j] = v.x;
+                if (j + 1 < NV) bs[j + 1] = v.y;
+                if (j + 2 < NV) bs[j + 2] = v.z;
+                if (j + 3 < NV) bs[j + 3] = v.w;
+            }
+        } else {
+            bs[j] = a.bias ? a.bias[c0 + j] : 0.f;
+        }
     }
     const int rend = (blockIdx.y + 1) * kConvReqs < a.n ? (blockIdx.y + 1) * kConvReqs : a.n;
+    if constexpr (NV * sizeof(T) == 16 && H > 0) {
+        // 16-byte units: the loads of kConvBatchReqs requests are all issued before
+        // any of their stores (the slots are distinct, so no store aliases a load),
+        // so a thread waits on memory once per batch instead of once per request
+        for (int rb = blockIdx.y * kConvReqs; rb < rend; rb += kConvBatchReqs) {
+            int slot[kConvBatchReqs];
+            uint4 xu[kConvBatchReqs], wu[kConvBatchReqs][H];
+#pragma unroll
+            for (int q = 0; q < kConvBatchReqs; ++q) {
+                const int r = rb + q;
+                slot[q] = r < rend ? (a.idx ? a.idx[r] : r) : -1;
+            }
+#pragma unroll
+            for (int q = 0; q < kConvBatchReqs; ++q) {
+                if (slot[q] >= 0 && slot[q] < a.n_slots) {
+                    xu[q] = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)(rb + q) * a.C + c0));
+                    const uint4* sp =
+                        reinterpret_cast<const uint4*>(state + ((int64_t)slot[q] * a.C + c0) * H);
+#pragma unroll
+                    for (int u = 0; u < H; ++u) wu[q][u] = sp[u];
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < kConvBatchReqs; ++q) {
+                const int r = rb + q;
+                if (r >= rend) break;
+                float o[NV];
+                if (slot[q] < 0 || slot[q] >= a.n_slots) {
+                    if (slot[q] >= a.n_slots) record_status(GDN_ERR_INVALID_ARG);
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) o[j] = 0.f;
+                    conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
+                    continue;
+                }
+                const T* xe = reinterpret_cast<const T*>(&xu[q]);
+                uint4 nu[H];
+#pragma unroll
+                for (int j = 0; j < NV; ++j) {
+                    const float xc = to_f32(xe[j]);
+                    float acc = bs[j];
+#pragma unroll
+                    for (int i = 0; i < H; ++i) {
+                        const int e = j * H + i;
+                        acc = fmaf(wt[i][j], to_f32(reinterpret_cast<const T*>(&wu[q][e / NV])[e % NV]),
+                                   acc);
+                    }
+                    acc = fmaf(wt[H][j], xc, acc);
+                    o[j] = ACT ? conv_silu(acc) : acc;
+#pragma unroll
+                    for (int i = 0; i < H; ++i) {
+                        const int e = j * H + i;
+                        const T v = (i + 1 < H)
+                                        ? reinterpret_cast<const T*>(&wu[q][(e + 1) / NV])[(e + 1) % NV]
+                                        : xe[j];
+                        reinterpret_cast<T*>(&nu[e / NV])[e % NV] = v;
+                    }
+                }
+                conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
+                uint4* sp = reinterpret_cast<uint4*>(state + ((int64_t)slot[q] * a.C + c0) * H);
+#pragma unroll
+                for (int u = 0; u < H; ++u) sp[u] = nu[u];
+            }
+        }
+        return;
+    }
     for (int r = blockIdx.y * kConvReqs; r < rend; ++r) {
         const int slot = a.idx ? a.idx[r] : r;
         float o[NV];
