@@ -244,31 +244,4 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int32_t* __restric
     }
 }
 
-// Exclusive prefix sum of the sequences' chunk counts ceil(len / C):
-// off[s] = chunks before sequence s, off[n_seq] = the batch's total.  One block.
-__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* __restrict__ cu,
-                                                             int n_seq, int C,
-                                                             int32_t* __restrict__ off) {
-    __shared__ int32_t part[1024];
-    const int per = (n_seq + 1023) / 1024;
-    const int b = threadIdx.x * per;
-    const int e = b + per < n_seq ? b + per : n_seq;
-    int32_t sum = 0;
-    for (int i = b; i < e; ++i) sum += (cu[i + 1] - cu[i] + C - 1) / C;
-    part[threadIdx.x] = sum;
-    __syncthreads();
-    for (int d = 1; d < 1024; d <<= 1) {  // inclusive scan of the per-thread sums
-        const int32_t v = threadIdx.x >= d ? part[threadIdx.x - d] : 0;
-        __syncthreads();
-        part[threadIdx.x] += v;
-        __syncthreads();
-    }
-    int32_t run = part[threadIdx.x] - sum;
-    for (int i = b; i < e; ++i) {
-        off[i] = run;
-        run += (cu[i + 1] - cu[i] + C - 1) / C;
-    }
-    if (threadIdx.x == 1023) off[n_seq] = part[1023];
-}
-
 }  // namespace gdn

@@ -138,11 +138,14 @@ enum : int {
 };
 static_assert(B_SLOTDONE + NPREP <= NBARS, "barrier slots");
 
-// Launch forms of the kernel: one cluster of (prep, chain) per (sequence,
-// head), or the two roles as separate launches that hand the slot images over
-// through global memory: the prep launch spreads every (chunk, head) of the
-// batch over all SMs, the chain launch runs one CTA per (sequence, head).
-enum : int { kFused = 0, kPrep = 1, kChain = 2 };
+// Launch forms of the kernel.  kFused: one cluster of (prep, chain) per
+// (sequence, head), the slot images pushed into the chain CTA with
+// cluster bulk copies.  kPersist (dense batches): one cooperative launch over
+// every SM; CTAs [0, n_chain) carry one chain each, the others build the
+// images of every (chunk, head) of the batch in chunk-major order, write each
+// to global memory and publish it with a ready flag, which the chain CTA waits
+// for (bounded) before it bulk-loads the image into its slot.
+enum : int { kFused = 0, kPersist = 1 };
 constexpr uint32_t kScalBytes = (uint32_t)sizeof(ChainScal);
 
 struct Params {
@@ -157,14 +160,14 @@ struct Params {
     float scale;
     void* o;
     float* hT;
-    // split launches: images [n_img][SZ_SLOT] then gate factors [n_img][kScalBytes],
-    // image (gi * H + head) for chunk gi of the batch (gi = choff[seq] + c, or
-    // seq * nch_dense + c for a dense batch)
+    // persistent form: images [n_img][SZ_SLOT] then gate factors [n_img][kScalBytes];
+    // image gi * H + head for chunk gi = seq * nch_dense + c of the dense batch
     uint8_t* img;
-    const int32_t* choff;  // [n_seq + 1] chunk offsets of a packed batch, or null
     int nch_dense;
     int n_seq;
     int64_t n_img;
+    uint32_t* ready;  // [n_img] image ready flags (zeroed before the launch)
+    int n_chain;      // CTAs carrying chains
 };
 
 // Bounded wait that honours the CTA's abort flag.  `cluster` selects
@@ -318,14 +321,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
     uint32_t* misc = reinterpret_cast<uint32_t*>(base + OFF_MISC);
     volatile uint32_t* abort_flag = misc + 1;
 
-    const uint32_t rank = MODE == kFused ? tc::cluster_ctarank() : MODE == kPrep ? 0u : 1u;
+    const uint32_t rank = MODE == kFused ? tc::cluster_ctarank()
+                                         : (blockIdx.x < (unsigned)p.n_chain ? 1u : 0u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = p.H;
-    // the (sequence, head) of this cluster or chain CTA (the prep launch takes
-    // its (chunk, head) jobs from a strided list instead)
+    // the (sequence, head) of this cluster or chain CTA (persistent prep CTAs
+    // take their (chunk, head) jobs from a strided list instead)
     int head = 0, seq = 0, nch = 0;
     int64_t cs = 0, ce = 0;
-    if (MODE != kPrep) {
+    if (MODE == kFused || rank == 1) {
         const int sh = MODE == kFused ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
         head = sh % H;
         const int slot = sh / H;
@@ -394,9 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 int head;
                 int64_t t0, ce, gi;
             };
-            const int64_t njobs = MODE == kFused ? 0
-                                  : p.choff   ? (int64_t)p.choff[p.n_seq] * H
-                                              : (int64_t)p.n_seq * p.nch_dense * H;
+            const int64_t chains = (int64_t)p.n_seq * H;
+            const int64_t njobs = MODE == kFused ? 0 : chains * p.nch_dense;
             auto job_at = [&](int k, Job& jb) -> bool {
                 if constexpr (MODE == kFused) {
                     const int c = pg + k * NPREP;
@@ -407,28 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     jb.gi = 0;
                     return true;
                 } else {
-                    const int64_t j =
-                        (int64_t)blockIdx.x * NPREP + pg + (int64_t)k * gridDim.x * NPREP;
+                    // chunk-major over the (dense) batch's chains, so every chain's
+                    // chunk c is built before any chain's chunk c + 1
+                    const int pb = (int)blockIdx.x - p.n_chain, npb = (int)gridDim.x - p.n_chain;
+                    const int64_t j = (int64_t)pb * NPREP + pg + (int64_t)k * npb * NPREP;
                     if (j >= njobs) return false;
-                    const int64_t gi = j / H;
-                    jb.head = (int)(j - gi * H);
-                    jb.gi = gi;
-                    if (p.choff) {
-                        int lo = 0, hi = p.n_seq - 1;  // last sequence with choff <= gi
-                        while (lo < hi) {
-                            const int mid = (lo + hi + 1) >> 1;
-                            if (p.choff[mid] <= gi)
-                                lo = mid;
-                            else
-                                hi = mid - 1;
-                        }
-                        jb.t0 = p.cu[lo] + (int64_t)C * (gi - p.choff[lo]);
-                        jb.ce = p.cu[lo + 1];
-                    } else {
-                        const int64_t sq = gi / p.nch_dense;
-                        jb.t0 = sq * p.T + (int64_t)C * (gi - sq * p.nch_dense);
-                        jb.ce = (sq + 1) * p.T;
-                    }
+                    const int64_t c = j / chains, ch = j - c * chains;
+                    const int64_t sq = ch / H;
+                    jb.head = (int)(ch - sq * H);
+                    jb.gi = sq * p.nch_dense + c;
+                    jb.t0 = sq * p.T + (int64_t)C * c;
+                    jb.ce = (sq + 1) * p.T;
                     return true;
                 }
             };
@@ -651,6 +643,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                         issue_load(jn);
                         ++loads;
                     }
+                    if constexpr (MODE == kPersist) {
+                        // publish: the image's writes complete, then the ready flag
+                        tc::bulk_wait0();
+                        tc::fence_proxy_async_global();
+                        tc::st_release_gpu_u32(p.ready + jb.gi * H + hd, 1u);
+                    }
                 }
                 jb = jn;
                 have = more;
@@ -680,15 +678,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 // TMA warp: K, V and Q tiles (two buffers each, buffer c & 1) as their
                 // buffers fall free, and the slots back to the prep CTA once consumed
                 const uint32_t r_free0 = MODE == kFused ? tc::mapa(smem_u32(&bars[B_FREE]), 0) : 0u;
-                // split launches: this chain's images in global memory
-                const int64_t gi0 = MODE == kFused ? 0
-                                    : p.choff ? (int64_t)p.choff[seq]
-                                              : (int64_t)seq * p.nch_dense;
+                // persistent form: this chain's images in global memory
+                const int64_t gi0 = MODE == kFused ? 0 : (int64_t)seq * p.nch_dense;
                 int last_img = -1;
                 auto load_img = [&](int c) {
                     if (*abort_flag) return;
                     const int j = c % NPREP;
                     const int64_t ii = (gi0 + c) * H + head;
+                    if constexpr (MODE == kPersist) {
+                        // wait (bounded) for the prep CTAs to publish this image
+                        uint32_t i = 0;
+                        while (tc::ld_acquire_gpu_u32(p.ready + ii) == 0u) {
+                            if (++i == kPolls || *abort_flag) {
+                                if (!*abort_flag) {
+                                    *abort_flag = 1u;
+                                    record_status(GDN_ERR_TIMEOUT);
+                                }
+                                return;
+                            }
+                        }
+                        tc::fence_proxy_async_global();
+                    }
                     tc::mbar_arrive_expect_tx(&bars[B_TPF + j], kSlotTx);
                     tc::bulk_g2s(sbase + C_OFF_SL + j * SZ_SLOT, p.img + ii * SZ_SLOT, SZ_SLOT,
                                  &bars[B_TPF + j]);
@@ -719,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     load(0, c);
                     load(2, c);
                 }
-                if (MODE == kChain)
+                if (MODE == kPersist)
                     for (int c = 0; c < NPREP && c < nch; ++c) load_img(c);
                 for (int c = 0; c < nch; ++c) {
                     const uint32_t ph = (c >> 1) & 1;
@@ -992,15 +1002,13 @@ inline bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t co
 }  // namespace tcf
 
 // Launches the kernel: with `img` null, one cluster of two CTAs per (sequence,
-// head); otherwise the prep launch over every (chunk, head) of the batch (one
-// CTA per SM, a strided job list) and then the chain launch, one CTA per
-// (sequence, head), with the slot images passed through `img` (n_img images
-// and their gate factors; `choff` the packed batch's chunk offsets or null).
-// Returns 0 on success, 1 when the tensor maps could not be built, 2 on a
-// launch error.
+// head); otherwise (a dense batch) the persistent form, one cooperative launch
+// of one CTA per SM, with the slot images and their ready flags in `img` /
+// `ready` (n_img of each).  Returns 0 on success, 1 when the tensor maps could
+// not be built, 2 on a launch error.
 inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cudaStream_t st,
-                           uint8_t* img = nullptr, const int32_t* choff = nullptr,
-                           int64_t n_img = 0, int n_sms = 148) {
+                           uint8_t* img = nullptr, uint32_t* ready = nullptr, int64_t n_img = 0,
+                           int n_sms = 148) {
     tcf::Params p;
     memset(&p, 0, sizeof(p));
     const uint64_t cols = (uint64_t)a.H * 128;
@@ -1020,45 +1028,44 @@ inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cuda
     p.o = a.o;
     p.hT = a.hT;
     p.img = img;
-    p.choff = choff;
     p.nch_dense = a.cu_seqlens ? 0 : (int)((a.T + tcf::C - 1) / tcf::C);
     p.n_seq = a.n_seq;
     p.n_img = n_img;
+    p.ready = ready;
+    const bool persist = img && ready && !a.cu_seqlens;
     using KernFn = void (*)(tcf::Params);
-    KernFn kfused = obf16 ? tcf::chunk_fwd_tc_kernel<true, tcf::kFused>
-                          : tcf::chunk_fwd_tc_kernel<false, tcf::kFused>;
-    KernFn kprep = tcf::chunk_fwd_tc_kernel<false, tcf::kPrep>;
-    KernFn kchain = obf16 ? tcf::chunk_fwd_tc_kernel<true, tcf::kChain>
-                          : tcf::chunk_fwd_tc_kernel<false, tcf::kChain>;
-    for (KernFn k : {kfused, kprep, kchain})
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tcf::SMEM_BYTES) != cudaSuccess)
-            return 2;
+    KernFn kern = persist ? (obf16 ? tcf::chunk_fwd_tc_kernel<true, tcf::kPersist>
+                                   : tcf::chunk_fwd_tc_kernel<false, tcf::kPersist>)
+                          : (obf16 ? tcf::chunk_fwd_tc_kernel<true, tcf::kFused>
+                                   : tcf::chunk_fwd_tc_kernel<false, tcf::kFused>);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tcf::SMEM_BYTES) != cudaSuccess)
+        return 2;
     const int64_t chains = (int64_t)a.n_seq * a.H;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.blockDim = dim3(tcf::kThreads, 1, 1);
     cfg.dynamicSmemBytes = tcf::SMEM_BYTES;
     cfg.stream = st;
-    if (!img) {
+    cudaLaunchAttribute attr[1];
+    if (persist) {
+        // the chains on CTAs [0, chains), the prep on every other SM; all CTAs
+        // resident at once (cooperative), since chain CTAs wait on prep CTAs
+        p.n_chain = (int)chains;
+        if (cudaMemsetAsync(ready, 0, (size_t)n_img * 4, st) != cudaSuccess) return 2;
+        cfg.gridDim = dim3((unsigned)n_sms, 1, 1);
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
         cfg.gridDim = dim3((unsigned)(chains * 2), 1, 1);
-        cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kfused, p) != cudaSuccess) return 2;
-        return 0;
     }
-    // prep: enough CTAs for every job, at most one per SM
-    const int64_t jobs = n_img;  // an upper bound of the batch's (chunk, head) count
-    const int64_t want = (jobs + tcf::NPREP - 1) / tcf::NPREP;
-    cfg.gridDim = dim3((unsigned)(want < n_sms ? want : n_sms), 1, 1);
-    if (cudaLaunchKernelEx(&cfg, kprep, p) != cudaSuccess) return 2;
-    cfg.gridDim = dim3((unsigned)chains, 1, 1);
-    if (cudaLaunchKernelEx(&cfg, kchain, p) != cudaSuccess) return 2;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return 2;
     return 0;
 }
 

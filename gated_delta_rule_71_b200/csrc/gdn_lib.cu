@@ -67,20 +67,21 @@ constexpr size_t kSimtSmemMax = 227 * 1024;
 
 size_t ws_schedule_bytes(int n_seq) { return ((size_t)n_seq * 4 + 255) / 256 * 256; }
 
-// Workspace of gdn_chunk_fwd: [schedule | chunk offsets | slot images | gate
-// factors].  The images (one per (chunk, head), bf16 K = V = 128 only) let the
-// tensor-core path run as two launches; without room for them it runs fused.
+// Workspace of gdn_chunk_fwd: [packed-batch schedule | slot images | gate
+// factors | image ready flags].  The images (one per (chunk, head); bf16,
+// K = V = 128) let a dense batch run the tensor-core path as one persistent
+// launch; without room for them it runs as clusters.
 struct ChunkWs {
-    size_t off_choff, off_img, total;
+    size_t off_img, off_ready, total;
     int64_t n_img;
 };
 ChunkWs chunk_ws_layout(int n_seq, int64_t T_total, int H, bool images) {
     ChunkWs L;
-    L.off_choff = ws_schedule_bytes(n_seq);
-    L.off_img = (L.off_choff + ((size_t)n_seq + 1) * 4 + 1023) / 1024 * 1024;
+    const size_t sched = ws_schedule_bytes(n_seq);
+    L.off_img = (sched + 1023) / 1024 * 1024;
     L.n_img = images ? ((T_total + 63) / 64 + n_seq) * (int64_t)H : 0;
-    L.total = images ? L.off_img + (size_t)L.n_img * (gdn::tcf::SZ_SLOT + gdn::tcf::kScalBytes)
-                     : L.off_choff;
+    L.off_ready = L.off_img + (size_t)L.n_img * (gdn::tcf::SZ_SLOT + gdn::tcf::kScalBytes);
+    L.total = images ? L.off_ready + (size_t)L.n_img * 4 : sched;
     return L;
 }
 
@@ -279,19 +280,18 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype 
         const int64_t T_total = cu_seqlens ? T : (int64_t)B * T;
         const ChunkWs L = chunk_ws_layout(n_seq, T_total, H, true);
         uint8_t* img = nullptr;
-        int32_t* choff = nullptr;
-        if (workspace && aligned16(workspace) && ws_bytes >= L.total) {
+        uint32_t* ready = nullptr;
+        const int sms = num_sms();
+        // a dense batch whose chains leave at least a third of the SMs to the
+        // prep runs as one persistent launch (when the workspace holds the images)
+        if (!cu_seqlens && workspace && aligned16(workspace) && ws_bytes >= L.total &&
+            (int64_t)n_seq * H * 3 <= (int64_t)sms * 2) {
             uint8_t* ws = static_cast<uint8_t*>(workspace);
             img = ws + L.off_img;
-            if (cu_seqlens) {
-                choff = reinterpret_cast<int32_t*>(ws + L.off_choff);
-                gdn::chunk_offsets_kernel<<<1, 1024, 0, st>>>(cu_seqlens, n_seq, gdn::tcf::C, choff);
-                gdn_status s = launch_check();
-                if (s != GDN_OK) return s;
-            }
+            ready = reinterpret_cast<uint32_t*>(ws + L.off_ready);
         }
-        const int rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st, img, choff,
-                                            L.n_img, num_sms());
+        const int rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st, img, ready,
+                                            L.n_img, sms);
         if (rc == 1) return GDN_ERR_UNSUPPORTED;
         if (rc == 2) return cuda_check(cudaGetLastError() != cudaSuccess ? cudaErrorInvalidValue
                                                                          : cudaErrorInvalidValue);
