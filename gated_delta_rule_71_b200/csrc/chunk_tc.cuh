@@ -138,6 +138,16 @@ enum : int {
 };
 static_assert(B_SLOTDONE + NPREP <= NBARS, "barrier slots");
 
+// Launch forms of the kernel.  kFused: one cluster of (prep, chain) per
+// (sequence, head), the slot images pushed into the chain CTA with
+// cluster bulk copies.  kPersist (dense batches): one cooperative launch over
+// every SM; CTAs [0, n_chain) carry one chain each, the others build the
+// images of every (chunk, head) of the batch in chunk-major order, write each
+// to global memory and publish it with a ready flag, which the chain CTA waits
+// for (bounded) before it bulk-loads the image into its slot.
+enum : int { kFused = 0, kPersist = 1 };
+constexpr uint32_t kScalBytes = (uint32_t)sizeof(ChainScal);
+
 struct Params {
     CUtensorMap tm_q, tm_k, tm_v, tm_o;  // tm_o: fp32 output, 32 x 64 boxes
     const float* g;
@@ -150,6 +160,14 @@ struct Params {
     float scale;
     void* o;
     float* hT;
+    // persistent form: images [n_img][SZ_SLOT] then gate factors [n_img][kScalBytes];
+    // image gi * H + head for chunk gi = seq * nch_dense + c of the dense batch
+    uint8_t* img;
+    int nch_dense;
+    int n_seq;
+    int64_t n_img;
+    uint32_t* ready;  // [n_img] image ready flags (zeroed before the launch)
+    int n_chain;      // CTAs carrying chains
 };
 
 // Bounded wait that honours the CTA's abort flag.  `cluster` selects
@@ -292,7 +310,7 @@ __device__ __forceinline__ void invert_unit_lower(const float* Af, float* Tf, fl
 }
 
 
-template <bool OBF16>
+template <bool OBF16, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -303,22 +321,28 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
     uint32_t* misc = reinterpret_cast<uint32_t*>(base + OFF_MISC);
     volatile uint32_t* abort_flag = misc + 1;
 
-    const uint32_t rank = tc::cluster_ctarank();
+    const uint32_t rank = MODE == kFused ? tc::cluster_ctarank()
+                                         : (blockIdx.x < (unsigned)p.n_chain ? 1u : 0u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = p.H;
-    const int sh = blockIdx.x >> 1;
-    const int head = sh % H;
-    const int slot = sh / H;
-    const int seq = p.order ? p.order[slot] : slot;
-    int64_t cs, ce;
-    if (p.cu) {
-        cs = p.cu[seq];
-        ce = p.cu[seq + 1];
-    } else {
-        cs = (int64_t)seq * p.T;
-        ce = cs + p.T;
+    // the (sequence, head) of this cluster or chain CTA (persistent prep CTAs
+    // take their (chunk, head) jobs from a strided list instead)
+    int head = 0, seq = 0, nch = 0;
+    int64_t cs = 0, ce = 0;
+    if (MODE == kFused || rank == 1) {
+        const int sh = MODE == kFused ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+        head = sh % H;
+        const int slot = sh / H;
+        seq = p.order ? p.order[slot] : slot;
+        if (p.cu) {
+            cs = p.cu[seq];
+            ce = p.cu[seq + 1];
+        } else {
+            cs = (int64_t)seq * p.T;
+            ce = cs + p.T;
+        }
+        nch = (int)((ce - cs + C - 1) / C);
     }
-    const int nch = (int)((ce - cs + C - 1) / C);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBARS; ++i)
@@ -329,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         // chain: arm the slot barriers for the first images before the prep CTA
         // can start a copy (it waits at the cluster barrier below)
-        if (rank == 1)
+        if (MODE == kFused && rank == 1)
             for (int i = 0; i < NPREP; ++i)
                 tc::mbar_arrive_expect_tx(&bars[B_TPF + i], SZ_SLOT + (uint32_t)sizeof(ChainScal));
     }
@@ -337,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
     if (warp == 0) tc::tmem_alloc(&misc[0], ncols);
     tc::tc_before_sync();
     __syncthreads();
-    tc::cluster_sync();  // both CTAs' barriers initialised before any remote arrive
+    if (MODE == kFused) tc::cluster_sync();  // both CTAs' barriers initialised before any remote arrive
     tc::tc_after_sync();
     const uint32_t tmem = misc[0];
 
@@ -359,35 +383,72 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             uint64_t* sfree = &bars[B_FREE + pg];
             const uint32_t tcol = tmem + 128u * pg;  // S_kk (64 columns), then W (128)
             // this warpgroup's slot in the chain CTA, and the staged gate factors
-            const uint32_t r_sl = tc::mapa(sbase + C_OFF_SL + pg * SZ_SLOT, 1);
-            const uint32_t r_sc = tc::mapa(sbase + C_OFF_SC + pg * (uint32_t)sizeof(ChainScal), 1);
-            const uint32_t r_tpf = tc::mapa(smem_u32(&bars[B_TPF + pg]), 1);
+            uint32_t r_sl = 0, r_sc = 0, r_tpf = 0;
+            if (MODE == kFused) {
+                r_sl = tc::mapa(sbase + C_OFF_SL + pg * SZ_SLOT, 1);
+                r_sc = tc::mapa(sbase + C_OFF_SC + pg * (uint32_t)sizeof(ChainScal), 1);
+                r_tpf = tc::mapa(smem_u32(&bars[B_TPF + pg]), 1);
+            }
             ChainScal* cst = reinterpret_cast<ChainScal*>(base + P_OFF_CS + pg * 528);
             const uint32_t cst_u32 = sbase + P_OFF_CS + pg * 528;
             const uint32_t idS = tc::idesc_bf16(128, 64, 0, 0);
             const uint32_t idW = tc::idesc_bf16(128, 128, 0, 1);
-            auto issue_load = [&](int c) {
-                const int y = (int)(cs + (int64_t)C * c);
-                tc::mbar_arrive_expect_tx(full, SZ_KQ);
-                tc::tma_load_2d(kq_p + 0, &p.tm_k, head * KD + 0, y, full);
-                tc::tma_load_2d(kq_p + 8192, &p.tm_q, head * KD + 0, y, full);
-                tc::tma_load_2d(kq_p + 16384, &p.tm_k, head * KD + 64, y, full);
-                tc::tma_load_2d(kq_p + 24576, &p.tm_q, head * KD + 64, y, full);
+            // this warpgroup's k-th job: chunk c (first row t0, sequence end ce) of head
+            struct Job {
+                int head;
+                int64_t t0, ce, gi;
             };
-            int last_loaded = -1;
-            if (pt == 0 && pg < nch) {
+            const int64_t chains = (int64_t)p.n_seq * H;
+            const int64_t njobs = MODE == kFused ? 0 : chains * p.nch_dense;
+            auto job_at = [&](int k, Job& jb) -> bool {
+                if constexpr (MODE == kFused) {
+                    const int c = pg + k * NPREP;
+                    if (c >= nch) return false;
+                    jb.head = head;
+                    jb.t0 = cs + (int64_t)C * c;
+                    jb.ce = ce;
+                    jb.gi = 0;
+                    return true;
+                } else {
+                    // chunk-major over the (dense) batch's chains, so every chain's
+                    // chunk c is built before any chain's chunk c + 1
+                    const int pb = (int)blockIdx.x - p.n_chain, npb = (int)gridDim.x - p.n_chain;
+                    const int64_t j = (int64_t)pb * NPREP + pg + (int64_t)k * npb * NPREP;
+                    if (j >= njobs) return false;
+                    const int64_t c = j / chains, ch = j - c * chains;
+                    const int64_t sq = ch / H;
+                    jb.head = (int)(ch - sq * H);
+                    jb.gi = sq * p.nch_dense + c;
+                    jb.t0 = sq * p.T + (int64_t)C * c;
+                    jb.ce = (sq + 1) * p.T;
+                    return true;
+                }
+            };
+            auto issue_load = [&](const Job& jb) {
+                const int y = (int)jb.t0;
+                tc::mbar_arrive_expect_tx(full, SZ_KQ);
+                tc::tma_load_2d(kq_p + 0, &p.tm_k, jb.head * KD + 0, y, full);
+                tc::tma_load_2d(kq_p + 8192, &p.tm_q, jb.head * KD + 0, y, full);
+                tc::tma_load_2d(kq_p + 16384, &p.tm_k, jb.head * KD + 64, y, full);
+                tc::tma_load_2d(kq_p + 24576, &p.tm_q, jb.head * KD + 64, y, full);
+            };
+            Job jb, jn;
+            bool have = job_at(0, jb);
+            int loads = 0;
+            if (pt == 0 && have) {
                 tc::prefetch_tmap(&p.tm_q);
                 tc::prefetch_tmap(&p.tm_k);
-                issue_load(pg);
-                last_loaded = pg;
+                issue_load(jb);
+                loads = 1;
             }
-            for (int c = pg, n = 0; c < nch; c += NPREP, ++n) {
-                const int64_t t0 = cs + (int64_t)C * c;
-                const int len = (int)((ce - t0) < C ? (ce - t0) : C);
+            for (int n = 0; have; ++n) {
+                const int64_t t0 = jb.t0;
+                const int len = (int)((jb.ce - t0) < C ? (jb.ce - t0) : C);
+                const int hd = jb.head;
                 float gv = 0.f, bv = 0.f;
                 if (pt < len) {
-                    gv = p.g[(t0 + pt) * H + head];
-                    bv = p.beta[(t0 + pt) * H + head];
+                    gv = p.g[(t0 + pt) * H + hd];
+                    bv = p.beta[(t0 + pt) * H + hd];
                 }
                 wait(full, n & 1, abort_flag);
                 if (pt == 0) {
@@ -562,23 +623,40 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 tc::fence_async_smem();
                 tc::tc_before_sync();
                 tc::named_bar(bid, 128);
+                const bool more = job_at(n + 1, jn);
                 if (pt == 0) {
-                    // hand the slot image to the chain CTA, then reuse the stage
-                    if (n >= 1) wait(sfree, (n - 1) & 1, abort_flag, true);
-                    tc::bulk_s2cluster(r_sl, kq, SZ_SLOT, r_tpf);
-                    tc::bulk_s2cluster(r_sc, cst_u32, (uint32_t)sizeof(ChainScal), r_tpf);
+                    // hand the slot image on (to the chain CTA, or to global memory),
+                    // then reuse the stage
+                    if constexpr (MODE == kFused) {
+                        if (n >= 1) wait(sfree, (n - 1) & 1, abort_flag, true);
+                        tc::bulk_s2cluster(r_sl, kq, SZ_SLOT, r_tpf);
+                        tc::bulk_s2cluster(r_sc, cst_u32, kScalBytes, r_tpf);
+                    } else {
+                        const int64_t ii = jb.gi * H + hd;
+                        tc::bulk_s2g(p.img + ii * SZ_SLOT, kq, SZ_SLOT);
+                        tc::bulk_s2g(p.img + p.n_img * SZ_SLOT + ii * kScalBytes, cst_u32,
+                                     kScalBytes);
+                    }
                     tc::bulk_commit();
                     tc::bulk_wait_read0();
-                    if (c + NPREP < nch) {
-                        issue_load(c + NPREP);
-                        last_loaded = c + NPREP;
+                    if (more && !*abort_flag) {
+                        issue_load(jn);
+                        ++loads;
+                    }
+                    if constexpr (MODE == kPersist) {
+                        // publish: the image's writes complete, then the ready flag
+                        tc::bulk_wait0();
+                        tc::fence_proxy_async_global();
+                        tc::st_release_gpu_u32(p.ready + jb.gi * H + hd, 1u);
                     }
                 }
+                jb = jn;
+                have = more;
             }
             if (pt == 0) {
                 // never leave with a copy or an MMA in flight
                 tc::bulk_wait0();
-                if (last_loaded >= 0) drain_wait(full, (last_loaded / NPREP) & 1);
+                if (loads > 0) drain_wait(full, (loads - 1) & 1);
                 if (*abort_flag) {
                     tc::mma_commit(&bars[B_DRAINP]);
                     drain_wait(&bars[B_DRAINP], 0);
@@ -599,7 +677,36 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             if (lane == 0) {
                 // TMA warp: K, V and Q tiles (two buffers each, buffer c & 1) as their
                 // buffers fall free, and the slots back to the prep CTA once consumed
-                const uint32_t r_free0 = tc::mapa(smem_u32(&bars[B_FREE]), 0);
+                const uint32_t r_free0 = MODE == kFused ? tc::mapa(smem_u32(&bars[B_FREE]), 0) : 0u;
+                // persistent form: this chain's images in global memory
+                const int64_t gi0 = MODE == kFused ? 0 : (int64_t)seq * p.nch_dense;
+                int last_img = -1;
+                auto load_img = [&](int c) {
+                    if (*abort_flag) return;
+                    const int j = c % NPREP;
+                    const int64_t ii = (gi0 + c) * H + head;
+                    if constexpr (MODE == kPersist) {
+                        // wait (bounded) for the prep CTAs to publish this image
+                        uint32_t i = 0;
+                        while (tc::ld_acquire_gpu_u32(p.ready + ii) == 0u) {
+                            if (++i == kPolls || *abort_flag) {
+                                if (!*abort_flag) {
+                                    *abort_flag = 1u;
+                                    record_status(GDN_ERR_TIMEOUT);
+                                }
+                                return;
+                            }
+                        }
+                        tc::fence_proxy_async_global();
+                    }
+                    tc::mbar_arrive_expect_tx(&bars[B_TPF + j], kSlotTx);
+                    tc::bulk_g2s(sbase + C_OFF_SL + j * SZ_SLOT, p.img + ii * SZ_SLOT, SZ_SLOT,
+                                 &bars[B_TPF + j]);
+                    tc::bulk_g2s(sbase + C_OFF_SC + j * kScalBytes,
+                                 p.img + p.n_img * SZ_SLOT + ii * kScalBytes, kScalBytes,
+                                 &bars[B_TPF + j]);
+                    last_img = c;
+                };
                 int last[3] = {-1, -1, -1};
                 auto load = [&](int kind, int c) {
                     if (*abort_flag) return;  // at most one copy in flight per buffer
@@ -622,6 +729,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     load(0, c);
                     load(2, c);
                 }
+                if (MODE == kPersist)
+                    for (int c = 0; c < NPREP && c < nch; ++c) load_img(c);
                 for (int c = 0; c < nch; ++c) {
                     const uint32_t ph = (c >> 1) & 1;
                     if (c + 2 < nch) {
@@ -631,14 +740,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     }
                     if (c + NPREP < nch) {
                         // re-arm the slot's barrier for the next image, then hand the
-                        // slot back to the prep CTA
+                        // slot back to the prep CTA (or fetch that image)
                         const int j = c % NPREP;
                         if (wait(&bars[B_SLOTDONE + j], (c / NPREP) & 1, abort_flag)) {
-                            tc::mbar_arrive_expect_tx(&bars[B_TPF + j], kSlotTx);
-                            tc::mbar_arrive_cluster(r_free0 + 8 * j);
+                            if constexpr (MODE == kFused) {
+                                tc::mbar_arrive_expect_tx(&bars[B_TPF + j], kSlotTx);
+                                tc::mbar_arrive_cluster(r_free0 + 8 * j);
+                            } else {
+                                load_img(c + NPREP);
+                            }
                         }
                     }
                 }
+                for (int c = last_img - NPREP + 1; c <= last_img; ++c)
+                    if (c >= 0) drain_wait(&bars[B_TPF + c % NPREP], (c / NPREP) & 1);
                 // never leave with a copy in flight
                 for (int kind = 0; kind < 3; ++kind) {
                     uint64_t* b0 = &bars[kind == 0 ? B_FULL : kind == 1 ? B_VF : B_QF];
@@ -847,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
     }
     tc::tc_before_sync();
     __syncthreads();
-    tc::cluster_sync();  // no CTA leaves while the other may still touch its memory
+    if (MODE == kFused) tc::cluster_sync();  // no CTA leaves while the other may still touch its memory
     tc::tc_after_sync();
     if (warp == 0) tc::tmem_dealloc(tmem, ncols);
 }
@@ -886,10 +1001,14 @@ inline bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t co
 
 }  // namespace tcf
 
-// Launches the fused kernel: one cluster of two CTAs per (sequence, head).
-// Returns 0 on success, 1 when the tensor maps could not be built, 2 on a
-// launch error.
-inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cudaStream_t st) {
+// Launches the kernel: with `img` null, one cluster of two CTAs per (sequence,
+// head); otherwise (a dense batch) the persistent form, one cooperative launch
+// of one CTA per SM, with the slot images and their ready flags in `img` /
+// `ready` (n_img of each).  Returns 0 on success, 1 when the tensor maps could
+// not be built, 2 on a launch error.
+inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cudaStream_t st,
+                           uint8_t* img = nullptr, uint32_t* ready = nullptr, int64_t n_img = 0,
+                           int n_sms = 148) {
     tcf::Params p;
     memset(&p, 0, sizeof(p));
     const uint64_t cols = (uint64_t)a.H * 128;
@@ -908,22 +1027,42 @@ inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cuda
     p.scale = a.scale;
     p.o = a.o;
     p.hT = a.hT;
-    const int64_t nb = (int64_t)a.n_seq * a.H * 2;
-    auto kern = obf16 ? tcf::chunk_fwd_tc_kernel<true> : tcf::chunk_fwd_tc_kernel<false>;
+    p.img = img;
+    p.nch_dense = a.cu_seqlens ? 0 : (int)((a.T + tcf::C - 1) / tcf::C);
+    p.n_seq = a.n_seq;
+    p.n_img = n_img;
+    p.ready = ready;
+    const bool persist = img && ready && !a.cu_seqlens;
+    using KernFn = void (*)(tcf::Params);
+    KernFn kern = persist ? (obf16 ? tcf::chunk_fwd_tc_kernel<true, tcf::kPersist>
+                                   : tcf::chunk_fwd_tc_kernel<false, tcf::kPersist>)
+                          : (obf16 ? tcf::chunk_fwd_tc_kernel<true, tcf::kFused>
+                                   : tcf::chunk_fwd_tc_kernel<false, tcf::kFused>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tcf::SMEM_BYTES) != cudaSuccess)
         return 2;
+    const int64_t chains = (int64_t)a.n_seq * a.H;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)nb, 1, 1);
     cfg.blockDim = dim3(tcf::kThreads, 1, 1);
     cfg.dynamicSmemBytes = tcf::SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    if (persist) {
+        // the chains on CTAs [0, chains), the prep on every other SM; all CTAs
+        // resident at once (cooperative), since chain CTAs wait on prep CTAs
+        p.n_chain = (int)chains;
+        if (cudaMemsetAsync(ready, 0, (size_t)n_img * 4, st) != cudaSuccess) return 2;
+        cfg.gridDim = dim3((unsigned)n_sms, 1, 1);
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        cfg.gridDim = dim3((unsigned)(chains * 2), 1, 1);
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return 2;

@@ -366,63 +366,63 @@ __global__ void __launch_bounds__(128) conv1d_update_kernel(const ConvUpdateArgs
                 for (int u = 0; u < H; ++u) sp[u] = nu[u];
             }
         }
-        return;
-    }
-    for (int r = blockIdx.y * kConvReqs; r < rend; ++r) {
-        const int slot = a.idx ? a.idx[r] : r;
-        float o[NV];
-        if (slot < 0 || slot >= a.n_slots) {
-            if (slot >= a.n_slots) record_status(GDN_ERR_INVALID_ARG);
+    } else {
+        for (int r = blockIdx.y * kConvReqs; r < rend; ++r) {
+            const int slot = a.idx ? a.idx[r] : r;
+            float o[NV];
+            if (slot < 0 || slot >= a.n_slots) {
+                if (slot >= a.n_slots) record_status(GDN_ERR_INVALID_ARG);
 #pragma unroll
-            for (int j = 0; j < NV; ++j) o[j] = 0.f;
+                for (int j = 0; j < NV; ++j) o[j] = 0.f;
+                conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
+                continue;
+            }
+            float xc[NV];
+            conv_load<T, NV>(x + (int64_t)r * a.C + c0, xc);
+            T* sp = state + ((int64_t)slot * a.C + c0) * H;  // NV*H contiguous values
+            if constexpr (NV * sizeof(T) == 16) {
+                // the window is H 16-byte units; element e = j*H + i sits in unit e / NV
+                uint4 wu[H > 0 ? H : 1], nu[H > 0 ? H : 1];
+#pragma unroll
+                for (int u = 0; u < H; ++u) wu[u] = reinterpret_cast<const uint4*>(sp)[u];
+#pragma unroll
+                for (int j = 0; j < NV; ++j) {
+                    float acc = bs[j];
+#pragma unroll
+                    for (int i = 0; i < H; ++i) {
+                        const int e = j * H + i;
+                        acc = fmaf(wt[i][j], to_f32(reinterpret_cast<const T*>(&wu[e / NV])[e % NV]), acc);
+                    }
+                    acc = fmaf(wt[H][j], xc[j], acc);
+                    o[j] = ACT ? conv_silu(acc) : acc;
+#pragma unroll
+                    for (int i = 0; i < H; ++i) {
+                        const int e = j * H + i;
+                        const T v = (i + 1 < H) ? reinterpret_cast<const T*>(&wu[(e + 1) / NV])[(e + 1) % NV]
+                                                : from_f32<T>(xc[j]);
+                        reinterpret_cast<T*>(&nu[e / NV])[e % NV] = v;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < H; ++u) reinterpret_cast<uint4*>(sp)[u] = nu[u];
+            } else {
+#pragma unroll
+                for (int j = 0; j < NV; ++j) {
+                    float win[H > 0 ? H : 1];
+#pragma unroll
+                    for (int i = 0; i < H; ++i) win[i] = to_f32(sp[j * H + i]);
+                    float acc = bs[j];
+#pragma unroll
+                    for (int i = 0; i < H; ++i) acc = fmaf(wt[i][j], win[i], acc);
+                    acc = fmaf(wt[H][j], xc[j], acc);
+                    o[j] = ACT ? conv_silu(acc) : acc;
+#pragma unroll
+                    for (int i = 0; i + 1 < H; ++i) sp[j * H + i] = from_f32<T>(win[i + 1]);
+                    if constexpr (H > 0) sp[j * H + H - 1] = from_f32<T>(xc[j]);
+                }
+            }
             conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
-            continue;
         }
-        float xc[NV];
-        conv_load<T, NV>(x + (int64_t)r * a.C + c0, xc);
-        T* sp = state + ((int64_t)slot * a.C + c0) * H;  // NV*H contiguous values
-        if constexpr (NV * sizeof(T) == 16) {
-            // the window is H 16-byte units; element e = j*H + i sits in unit e / NV
-            uint4 wu[H > 0 ? H : 1], nu[H > 0 ? H : 1];
-#pragma unroll
-            for (int u = 0; u < H; ++u) wu[u] = reinterpret_cast<const uint4*>(sp)[u];
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                float acc = bs[j];
-#pragma unroll
-                for (int i = 0; i < H; ++i) {
-                    const int e = j * H + i;
-                    acc = fmaf(wt[i][j], to_f32(reinterpret_cast<const T*>(&wu[e / NV])[e % NV]), acc);
-                }
-                acc = fmaf(wt[H][j], xc[j], acc);
-                o[j] = ACT ? conv_silu(acc) : acc;
-#pragma unroll
-                for (int i = 0; i < H; ++i) {
-                    const int e = j * H + i;
-                    const T v = (i + 1 < H) ? reinterpret_cast<const T*>(&wu[(e + 1) / NV])[(e + 1) % NV]
-                                            : from_f32<T>(xc[j]);
-                    reinterpret_cast<T*>(&nu[e / NV])[e % NV] = v;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < H; ++u) reinterpret_cast<uint4*>(sp)[u] = nu[u];
-        } else {
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                float win[H > 0 ? H : 1];
-#pragma unroll
-                for (int i = 0; i < H; ++i) win[i] = to_f32(sp[j * H + i]);
-                float acc = bs[j];
-#pragma unroll
-                for (int i = 0; i < H; ++i) acc = fmaf(wt[i][j], win[i], acc);
-                acc = fmaf(wt[H][j], xc[j], acc);
-                o[j] = ACT ? conv_silu(acc) : acc;
-#pragma unroll
-                for (int i = 0; i + 1 < H; ++i) sp[j * H + i] = from_f32<T>(win[i + 1]);
-                if constexpr (H > 0) sp[j * H + H - 1] = from_f32<T>(xc[j]);
-            }
-        }
-        conv_store<T, NV>(y + (int64_t)r * a.C + c0, o);
     }
 }
 

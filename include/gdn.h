@@ -91,8 +91,13 @@ gdn_status gdn_gate_prep(const float* a, const float* b, int64_t n_tok, int H, i
                          float* g, void* stream);
 
 /*
- * gdn_chunk_fwd_workspace_size -- bytes of device workspace gdn_chunk_fwd
- * needs for these sizes (0 for a dense batch).  The caller allocates it.
+ * gdn_chunk_fwd_workspace_size -- bytes of device workspace for gdn_chunk_fwd
+ * with these sizes.  The caller allocates it.  It holds the packed-batch
+ * schedule (int32 per sequence) and, for bf16 q/k/v with K = V = 128, one
+ * 33,296-byte WY image per (chunk, head) plus a 4-byte ready flag each
+ * ((ceil(T_total / 64) + n_seq) * H of them): with that room a dense batch
+ * runs the tensor-core kernel as one persistent cooperative launch, the prep
+ * on every SM not carrying a chain (see gdn_chunk_fwd).  0 when n_seq <= 0.
  */
 size_t gdn_chunk_fwd_workspace_size(int n_seq, int64_t T_total, int H, int K, int V,
                                     gdn_dtype qkv_dtype);
@@ -111,9 +116,15 @@ size_t gdn_chunk_fwd_workspace_size(int n_seq, int64_t T_total, int H, int K, in
  *   scale   : multiplies every output (o_t = scale * S_t q_t).
  *   o       : [B, T, H, V] of o_dtype (GDN_F32 or GDN_BF16), written.
  *   hT      : fp32 [n_seq, H, K, V] final states, written; NULL to skip.
- *   workspace / ws_bytes : device scratch of at least
- *             gdn_chunk_fwd_workspace_size(...) bytes (may be NULL when that
- *             is 0).  Its contents on entry do not matter.
+ *   workspace / ws_bytes : device scratch of gdn_chunk_fwd_workspace_size(...)
+ *             bytes.  Its contents on entry do not matter.  A packed batch
+ *             needs at least its schedule (4 * n_seq bytes, rounded up to 256);
+ *             a dense batch may pass NULL.  With less than the full size the
+ *             bf16 K = V = 128 path runs as one cluster of two CTAs per
+ *             (sequence, head); with the full size, a dense batch whose
+ *             n_seq * H chains fit in two thirds of the SMs runs as one
+ *             cooperative launch (chains on n_seq * H CTAs, the WY prep of
+ *             every (chunk, head) on the other SMs), which is faster.
  *   flags   : GDN_FLAG_* bits; 0 selects the fastest kernel for the dtype.
  * Supported: K, V in {32, 64, 128}.  bf16 q/k/v run on the tcgen05 tensor-core
  * kernel (bf16 operands, fp32 accumulation and fp32 state) when K = V = 128;
