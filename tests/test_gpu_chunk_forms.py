@@ -74,3 +74,17 @@ def test_persistent_form_in_cuda_graph(cuda_device):
     torch.cuda.synchronize()
     assert gdn.device_status() == 0
     assert torch.equal(o, o_ref) and torch.equal(hT, h_ref)
+
+
+def test_dense_batch_beyond_persistent_capacity(cuda_device):
+    # 7 x 16 = 112 chains: more than two thirds of the SMs, so even with the full
+    # workspace the launch falls back to the cluster form
+    w = I.small_chunk_workload(7, 150, 16, 128, 128, torch.bfloat16, h0=True, seed=333)
+    inp, d, beta, g = _prep(w, cuda_device)
+    full = torch.empty(gdn.chunk_fwd_workspace_size(7, 7 * 150, 16, 128, 128), dtype=torch.uint8,
+                       device=cuda_device)
+    o, hT = _call(d, g, beta, full)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    ro, rh = oracle.gdn_fwd(inp["q"], inp["k"], inp["v"], g.cpu(), beta.cpu(), h0=inp["h0"])
+    assert relerr(o.cpu(), ro) <= TOL_BF16 and relerr(hT.cpu(), rh) <= TOL_BF16
