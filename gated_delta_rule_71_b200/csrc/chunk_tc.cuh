@@ -762,9 +762,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 }
             }
         } else if (warp == 16) {
-            if (lane == 0) {
+            {
                 // MMA warp: the dependent products (U, dS) are issued as soon as their
-                // inputs are written; the output products fill the gaps
+                // inputs are written; the output products fill the gaps.  All 32 lanes
+                // run it and one elected lane issues each product (warp-uniform
+                // operands give a shorter issue sequence than a lone lane).
                 const uint32_t idU0 = tc::idesc_bf16(128, 64, 1, 0);
                 const uint32_t id1 = tc::idesc_bf16(128, 64, 0, 0) | tc::kNegateA;
                 const uint32_t idO = tc::idesc_bf16(128, 64, 0, 0);
@@ -772,65 +774,72 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 // U0 for chunk c: D_U = V^T Tb^T  (A = V tile MN-major, B = Tb K-major)
                 auto issue_u0 = [&](int c) {
                     wait(&bars[B_VF + (c & 1)], (c >> 1) & 1, abort_flag);
+                    __syncwarp();
                     wait(&bars[B_TPF + c % NPREP], (c / NPREP) & 1, abort_flag);
+                    __syncwarp();
                     tc::tc_after_sync();
                     const uint32_t vt = sbase + C_OFF_V + (c & 1) * SZ_T;
                     const uint32_t tb = sbase + C_OFF_SL + (c % NPREP) * SZ_SLOT + SL_TB;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16(tmem + C_COL_U, tc::sdesc_sw128(vt + kk * 2048, 8192, 1024),
+                        tc::mma_bf16_w(tmem + C_COL_U, tc::sdesc_sw128(vt + kk * 2048, 8192, 1024),
                                      tc::sdesc_sw128(tb + kk * 32, 16, 1024), idU0, kk > 0);
-                    tc::mma_commit(&bars[B_VFREE + (c & 1)]);
+                    tc::mma_commit_w(&bars[B_VFREE + (c & 1)]);
                 };
                 if (nch > 0) issue_u0(0);
                 for (int c = 0; c < nch; ++c) {
                     const uint32_t sl = sbase + C_OFF_SL + (c % NPREP) * SZ_SLOT;
                     wait(s4, c & 1, abort_flag);  // bf16 S of this chunk written
+                    __syncwarp();
                     tc::tc_after_sync();
                     // Ut^T = V^T Tb^T - S W^T
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_bf16_ts(tmem + C_COL_U, tmem + C_COL_SB + 8 * kk,
+                        tc::mma_bf16_ts_w(tmem + C_COL_U, tmem + C_COL_SB + 8 * kk,
                                         tc::sdesc_sw128(sl + SL_W + (kk >> 2) * 8192 + (kk & 3) * 32,
                                                         16, 1024),
                                         id1, 1);
-                    tc::mma_commit(mA);
+                    tc::mma_commit_w(mA);
                     // S Q^T for the output
                     wait(&bars[B_QF + (c & 1)], (c >> 1) & 1, abort_flag);
+                    __syncwarp();
                     tc::tc_after_sync();
                     const uint32_t qt = sbase + C_OFF_Q + (c & 1) * SZ_T;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_bf16_ts(tmem + C_COL_O1 + 64u * (c & 1), tmem + C_COL_SB + 8 * kk,
+                        tc::mma_bf16_ts_w(tmem + C_COL_O1 + 64u * (c & 1), tmem + C_COL_SB + 8 * kk,
                                         tc::sdesc_sw128(qt + (kk >> 2) * 8192 + (kk & 3) * 32, 16,
                                                         1024),
                                         idO, kk > 0);
-                    tc::mma_commit(&bars[B_QFREE + (c & 1)]);
+                    tc::mma_commit_w(&bars[B_QFREE + (c & 1)]);
                     wait(s2, c & 1, abort_flag);  // Ut^T, (w Ut)^T written; output(c-1) done
+                    __syncwarp();
                     wait(&bars[B_FULL + (c & 1)], (c >> 1) & 1, abort_flag);
+                    __syncwarp();
                     tc::tc_after_sync();
                     // dS = (w Ut)^T K
                     const uint32_t kt = sbase + C_OFF_K + (c & 1) * SZ_T;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16_ts(tmem + C_COL_DS, tmem + C_COL_WB + 8 * kk,
+                        tc::mma_bf16_ts_w(tmem + C_COL_DS, tmem + C_COL_WB + 8 * kk,
                                         tc::sdesc_sw128(kt + kk * 2048, 8192, 1024), id2, kk > 0);
-                    tc::mma_commit(mD);
-                    tc::mma_commit(&bars[B_KFREE + (c & 1)]);
+                    tc::mma_commit_w(mD);
+                    tc::mma_commit_w(&bars[B_KFREE + (c & 1)]);
                     // Ut^T P^T
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16_ts(tmem + C_COL_O2, tmem + C_COL_UB + 8 * kk,
+                        tc::mma_bf16_ts_w(tmem + C_COL_O2, tmem + C_COL_UB + 8 * kk,
                                         tc::sdesc_sw128(sl + SL_P + kk * 32, 16, 1024), idO,
                                         kk > 0);
-                    tc::mma_commit(mO);
-                    tc::mma_commit(&bars[B_SLOTDONE + c % NPREP]);
+                    tc::mma_commit_w(mO);
+                    tc::mma_commit_w(&bars[B_SLOTDONE + c % NPREP]);
                     // next chunk's U0 (D_U was read before s2)
                     if (c + 1 < nch) issue_u0(c + 1);
                 }
                 // never leave with an MMA in flight
-                tc::mma_commit(&bars[B_DRAIN]);
+                tc::mma_commit_w(&bars[B_DRAIN]);
                 drain_wait(&bars[B_DRAIN], 0);
+                __syncwarp();
             }
         } else {
             const int wg = warp >> 2, q = warp & 3;
