@@ -290,11 +290,23 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype 
             img = ws + L.off_img;
             ready = reinterpret_cast<uint32_t*>(ws + L.off_ready);
         }
-        const int rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st, img, ready,
-                                            L.n_img, sms);
+        int rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st, img, ready, L.n_img,
+                                      sms);
+        if (rc == 2 && ready) {
+            // the cooperative launch could not make every CTA resident (other work
+            // holding SMs): run the cluster form instead
+            const cudaError_t e = cudaGetLastError();
+            if (e == cudaErrorCooperativeLaunchTooLarge)
+                rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st, nullptr, nullptr, 0,
+                                          sms);
+            else
+                return cuda_check(e != cudaSuccess ? e : cudaErrorLaunchFailure);
+        }
         if (rc == 1) return GDN_ERR_UNSUPPORTED;
-        if (rc == 2) return cuda_check(cudaGetLastError() != cudaSuccess ? cudaErrorInvalidValue
-                                                                         : cudaErrorInvalidValue);
+        if (rc == 2) {
+            const cudaError_t e = cudaGetLastError();
+            return cuda_check(e != cudaSuccess ? e : cudaErrorLaunchFailure);
+        }
         return launch_check();
     }
 
