@@ -236,6 +236,51 @@ def cpu_baseline(inp, target_s=12.0):
                       f"({tok_heads} token-heads, {dt:.1f} s); tokens/s = token-heads/s / H"}
 
 
+# ---------------------------------------------------- other chunk workloads
+
+def time_chunk_workload(gdn, I, w, dev, stream, world, peaks, src, n_iter=20):
+    """Times gdn.chunk_fwd alone on one chunk workload at full size (inputs
+    resident in HBM, gates prepared once), with the roofline of its algorithmic
+    bytes; the per-call time is the mean over n_iter back-to-back calls."""
+    inp = I.chunk_inputs(w)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    B, T, H, K, V = w.B, w.T, w.H, w.K, w.V
+    n_seq = w.n_seq_varlen if w.n_seq_varlen else B
+    beta, g = gdn.gate_prep(d["a"], d["b"], d["A_log"], d["dt_bias"])
+    o = torch.empty(B, T, H, V, device=dev)
+    hT = torch.empty(n_seq, H, K, V, device=dev)
+    ws = torch.empty(max(1, gdn.chunk_fwd_workspace_size(n_seq, B * T, H, K, V, w.dtype)),
+                     dtype=torch.uint8, device=dev)
+
+    def call():
+        gdn.chunk_fwd(d["q"], d["k"], d["v"], g, beta, h0=d["h0"], cu_seqlens=d["cu_seqlens"],
+                      out=o, hT=hT, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_iter):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_iter
+    by, fl = chunk_algorithmic(B, T, H, K, V, n_seq, h0=w.h0)
+    ach = by / (ms * 1e-3) / 1e9
+    lens = None
+    if d["cu_seqlens"] is not None:
+        cu = inp["cu_seqlens"].tolist()
+        lens = [cu[i + 1] - cu[i] for i in range(n_seq)]
+    del d, o, hT, ws
+    return {"workload": w.name, "metric": "tokens/s", "value": B * T * world / (ms * 1e-3),
+            "ms_per_step": ms, "n_seq": n_seq, "lengths": lens, "calls_timed": n_iter,
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                         "algorithmic_bytes": by, "algorithmic_flops": fl,
+                         "peak_source": src}}
+
+
 # ------------------------------------------------------------------- ours
 
 def run_ours(args):
@@ -403,6 +448,13 @@ def run_ours(args):
         + pw.B * pw.H * pw.N * pw.P * 4
     pf_ach = pf_by / (pf_ms * 1e-3) / 1e9
 
+    # --- the packed variable-length batch and the long single sequence, each at full
+    # size (their own tokens/s and roofline; not part of the headline step)
+    extra = {}
+    for key, wl in (("varlen", I.VARLEN_8x32768), ("long", I.LONG_T131072)):
+        extra[key] = time_chunk_workload(gdn, I, wl, dev, stream, world, peaks, src,
+                                         n_iter=max(3, min(args.steps, 20)))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp)
@@ -441,6 +493,8 @@ def run_ours(args):
                                   "ms_per_step": upd_ms,
                                   "achieved_gbs": round(upd_by / (upd_ms * 1e-3) / 1e9, 1),
                                   "algorithmic_bytes": upd_by}},
+            "varlen": extra["varlen"],
+            "long": extra["long"],
             "gdp_prefill": {"workload": pw.name, "metric": "tokens/s",
                             "value": pf_rows * world / (pf_ms * 1e-3), "ms_per_step": pf_ms,
                             "path": "gdp_decode_prepare over the prompt, the chunked kernel over "

@@ -67,24 +67,6 @@ constexpr size_t kSimtSmemMax = 227 * 1024;
 
 size_t ws_schedule_bytes(int n_seq) { return ((size_t)n_seq * 4 + 255) / 256 * 256; }
 
-// Workspace of gdn_chunk_fwd: [packed-batch schedule | slot images | gate
-// factors | image ready flags].  The images (one per (chunk, head); bf16,
-// K = V = 128) let a dense batch run the tensor-core path as one persistent
-// launch; without room for them it runs as clusters.
-struct ChunkWs {
-    size_t off_img, off_ready, total;
-    int64_t n_img;
-};
-ChunkWs chunk_ws_layout(int n_seq, int64_t T_total, int H, bool images) {
-    ChunkWs L;
-    const size_t sched = ws_schedule_bytes(n_seq);
-    L.off_img = (sched + 1023) / 1024 * 1024;
-    L.n_img = images ? ((T_total + 63) / 64 + n_seq) * (int64_t)H : 0;
-    L.off_ready = L.off_img + (size_t)L.n_img * (gdn::tcf::SZ_SLOT + gdn::tcf::kScalBytes);
-    L.total = images ? L.off_ready + (size_t)L.n_img * 4 : sched;
-    return L;
-}
-
 }  // namespace
 
 namespace {
@@ -220,9 +202,11 @@ gdn_status gdn_gate_prep(const float* a, const float* b, int64_t n_tok, int H, i
 
 size_t gdn_chunk_fwd_workspace_size(int n_seq, int64_t T_total, int H, int K, int V,
                                     gdn_dtype qkv_dtype) {
+    (void)K;
+    (void)V;
+    (void)qkv_dtype;
     if (n_seq <= 0 || H < 1 || T_total < 0) return 0;
-    const bool images = gdn::kTcAvailable && qkv_dtype == GDN_BF16 && K == 128 && V == 128;
-    return chunk_ws_layout(n_seq, T_total, H, images).total;
+    return ws_schedule_bytes(n_seq);
 }
 
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype qkv_dtype,
@@ -278,30 +262,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, gdn_dtype 
         a.nvs = 2;
         a.VS = V / 2;
         const int64_t T_total = cu_seqlens ? T : (int64_t)B * T;
-        const ChunkWs L = chunk_ws_layout(n_seq, T_total, H, true);
-        uint8_t* img = nullptr;
-        uint32_t* ready = nullptr;
-        const int sms = num_sms();
-        // a dense batch whose chains leave at least a third of the SMs to the
-        // prep runs as one persistent launch (when the workspace holds the images)
-        if (!cu_seqlens && workspace && aligned16(workspace) && ws_bytes >= L.total &&
-            (int64_t)n_seq * H * 3 <= (int64_t)sms * 2) {
-            uint8_t* ws = static_cast<uint8_t*>(workspace);
-            img = ws + L.off_img;
-            ready = reinterpret_cast<uint32_t*>(ws + L.off_ready);
-        }
-        int rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st, img, ready, L.n_img,
-                                      sms);
-        if (rc == 2 && ready) {
-            // the cooperative launch could not make every CTA resident (other work
-            // holding SMs): run the cluster form instead
-            const cudaError_t e = cudaGetLastError();
-            if (e == cudaErrorCooperativeLaunchTooLarge)
-                rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st, nullptr, nullptr, 0,
-                                          sms);
-            else
-                return cuda_check(e != cudaSuccess ? e : cudaErrorLaunchFailure);
-        }
+        const int rc = gdn::launch_chunk_tc(a, T_total, o_dtype == GDN_BF16, st);
         if (rc == 1) return GDN_ERR_UNSUPPORTED;
         if (rc == 2) {
             const cudaError_t e = cudaGetLastError();

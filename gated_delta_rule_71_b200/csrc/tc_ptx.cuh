@@ -206,6 +206,113 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor split into its two 32-bit words: the low word holds the
+// start address and the leading-byte offset, the high word the stride-byte
+// offset (1024: eight 128-byte rows), the SM100 version bit and the 128-byte
+// swizzle.  Stepping a K-block is a constant add to the low word (no carry:
+// shared addresses stay below 2^18).
+__host__ __device__ constexpr uint32_t desc_hi_sw128() {
+    return (1024u >> 4) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t desc(uint32_t lo) {
+    return ((uint64_t)desc_hi_sw128() << 32) | lo;
+}
+// One thread's products with the accumulate flag fixed at compile time.
+template <int ACC>
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "n"(ACC)
+        : "memory");
+}
+template <int ACC>
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "n"(ACC)
+        : "memory");
+}
+
+// Warp-wide forms of the same: called by all 32 lanes of a converged warp, one
+// elected lane issues (on this part about 36 cycles per M=128, N=64 product
+// against about 60 from a lone lane).  Commits must come from the same elected
+// lane (mma_commit_w), since a commit tracks the issuing thread's products.
+template <int ACC>
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc) {
+    asm volatile(
+        "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "n"(ACC)
+        : "memory");
+}
+template <int ACC>
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                         uint32_t idesc) {
+    asm volatile(
+        "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "n"(ACC)
+        : "memory");
+}
+
+// Four or eight products in one issue sequence of a converged warp (one elected
+// lane): A = the tensor-memory columns a, a + 8, ... (16 bf16 each), B = the
+// shared-memory descriptors hi:b_lo[k], D accumulated (the first product
+// accumulates when ACC0 is set).
+template <int ACC0>
+__device__ __forceinline__ void mma_ts4_w(uint32_t d, uint32_t a, uint32_t b0, uint32_t b1,
+                                          uint32_t b2, uint32_t b3, uint32_t idesc) {
+    asm volatile(
+        "{\n .reg .pred e, p;\n .reg .b64 d0, d1, d2, d3;\n setp.ne.b32 p, %11, 0;\n"
+        " mov.b64 d0, {%3, %10};\n mov.b64 d1, {%4, %10};\n"
+        " mov.b64 d2, {%5, %10};\n mov.b64 d3, {%6, %10};\n"
+        " elect.sync _|e, 0xffffffff;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], d0, %2, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], d1, %2, 1;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], d2, %2, 1;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], d3, %2, 1;\n}\n" ::"r"(d),
+        "r"(a), "r"(idesc), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(a + 8), "r"(a + 16),
+        "r"(a + 24), "r"(desc_hi_sw128()), "n"(ACC0)
+        : "memory");
+}
+template <int ACC0>
+__device__ __forceinline__ void mma_ss4_w(uint32_t d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1, uint32_t b2,
+                                          uint32_t b3, uint32_t idesc) {
+    asm volatile(
+        "{\n .reg .pred e, p;\n .reg .b64 x0, x1, x2, x3, y0, y1, y2, y3;\n setp.ne.b32 p, %11, 0;\n"
+        " mov.b64 x0, {%1, %10};\n mov.b64 x1, {%2, %10};\n mov.b64 x2, {%3, %10};\n"
+        " mov.b64 x3, {%4, %10};\n mov.b64 y0, {%5, %10};\n mov.b64 y1, {%6, %10};\n"
+        " mov.b64 y2, {%7, %10};\n mov.b64 y3, {%8, %10};\n"
+        " elect.sync _|e, 0xffffffff;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], x0, y0, %9, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], x1, y1, %9, 1;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], x2, y2, %9, 1;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], x3, y3, %9, 1;\n}\n" ::"r"(d),
+        "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(idesc),
+        "r"(desc_hi_sw128()), "n"(ACC0)
+        : "memory");
+}
+
+// One elected lane of a converged warp (elect.sync).  Issuing tcgen05 products
+// and their commits inside `if (elect_one()) { ... }` lets the compiler see a
+// single active thread, which keeps each issue to a few instructions.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t e;
+    asm volatile(
+        "{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(e));
+    return e != 0;
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t accumulate) {
