@@ -66,18 +66,14 @@ constexpr uint32_t kIdleLimit = 1u << 27;  // loader: polls without progress bef
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---- the image of one chunk: three 64 x 64 bf16 tiles in the 128-byte swizzle
-// (each 1024-byte aligned) and the gate factors (separately, 528 bytes).  In the
-// prep CTA the tiles are contiguous [T' | Tb | P]; in a chain slot T' sits at
-// the start of a 16 KB area that later holds W^T, and the whole 32 KB slot
-// stages the chunk's fp32 output once its tiles are spent.
+// (each 1024-byte aligned) [T' | Tb | P], and the gate factors (528 bytes), which
+// the chain keeps in a ring of NFAC entries so that a slot can take the next
+// image as soon as its tiles are spent, while the factors are still read.
 constexpr uint32_t SL_TP = 0;       // T'  = T diag(beta gam)   [row r][col s]
-constexpr uint32_t SL_TB = 8192;    // Tb  = T diag(beta)           (prep image)
-constexpr uint32_t SL_P = 16384;    // P                           (prep image)
+constexpr uint32_t SL_TB = 8192;    // Tb  = T diag(beta)
+constexpr uint32_t SL_P = 16384;    // P' = scale P
 constexpr uint32_t SZ_TILES = 24576;
-constexpr uint32_t CS_WT = 0;       // chain slot: T', then W^T [128 keys][64 tokens]
-constexpr uint32_t CS_TB = 16384;   // chain slot: Tb
-constexpr uint32_t CS_P = 24576;    // chain slot: P
-constexpr uint32_t SZ_CSLOT = 32768;
+constexpr int NFAC = 2 * 3;         // gate-factor ring (two images per slot)
 struct ChainScal {
     float w[64];    // 2^(G2_L - G2)
     float gam[64];  // scale * 2^G2 (the output's inter-chunk factor)
@@ -111,13 +107,15 @@ static_assert(10 * 16 * XP * 4 <= SL_P, "inverse scratch fits below the P tile")
 
 // ---- shared memory, chain CTA
 constexpr uint32_t SZ_T = 16384;  // one K, V or Q tile: [2 halves][64 tokens][128 B]
-constexpr int NKB = 3, NVB = 3, NQB = 2;
+constexpr int NKB = 3, NVB = 2, NQB = 1;
 constexpr uint32_t C_OFF_K = 0;
 constexpr uint32_t C_OFF_V = C_OFF_K + NKB * SZ_T;
 constexpr uint32_t C_OFF_Q = C_OFF_V + NVB * SZ_T;
 constexpr uint32_t C_OFF_SL = C_OFF_Q + NQB * SZ_T;    // NPREP image slots
-constexpr uint32_t C_OFF_SC = C_OFF_SL + NPREP * SZ_CSLOT;  // NPREP x gate factors
-constexpr uint32_t C_END = C_OFF_SC + NPREP * kScalBytes;
+constexpr uint32_t C_OFF_WT = C_OFF_SL + NPREP * SZ_TILES;  // W^T bf16 [128 keys][64 tokens]
+constexpr uint32_t C_OFF_OUT = C_OFF_WT + 16384;           // fp32 output stage: 4 x [64][32]
+constexpr uint32_t C_OFF_SC = C_OFF_OUT + 32768;           // NFAC x gate factors
+constexpr uint32_t C_END = C_OFF_SC + NFAC * kScalBytes;
 
 constexpr uint32_t BODY = (P_END > C_END ? P_END : C_END);
 constexpr uint32_t OFF_BAR = (BODY + 15) & ~15u;
@@ -151,9 +149,10 @@ enum : int {
     C_VFREE = C_KFREE + NKB,       // [NVB] V buffer read (U0 done)
     C_QFREE = C_VFREE + NVB,       // [NQB] Q buffer read (S Q^T done)
     C_TPF = C_QFREE + NQB,         // [NPREP] slot filled (bulk-copy transactions from the prep CTA)
-    C_SLOTDONE = C_TPF + NPREP,    // [NPREP] slot free again (its staged output has been read out)
-    C_OUTRDY = C_SLOTDONE + NPREP, // [NPREP] chunk output staged in the slot (state-warp arrivals)
-    C_MA = C_OUTRDY + NPREP,       // Ut^T ready
+    C_SLOTDONE = C_TPF + NPREP,    // [NPREP] slot's tiles consumed (U^T P'^T commit)
+    C_OUTRDY = C_SLOTDONE + NPREP, // chunk output staged (state-warp arrivals)
+    C_STGFREE,                     // output stage read out by the TMA stores
+    C_MA,                          // Ut^T ready
     C_MD,                          // dS ready
     C_MO,                          // S Q^T and Ut^T P^T ready
     C_MW,                          // W^T ready
@@ -441,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
         for (int i = 0; i < NBARS; ++i) {
             uint32_t cnt = 1u;
             if (i == C_S2 || i == C_S4) cnt = (uint32_t)NSW;  // the state warps
-            if (i == C_OFREE || (i >= C_OUTRDY && i < C_OUTRDY + NPREP)) cnt = (uint32_t)NSW;
+            if (i == C_OFREE || i == C_OUTRDY) cnt = (uint32_t)NSW;
             mbar_init(&bars[i], cnt);
         }
         misc[1] = 0u;
@@ -480,8 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             uint64_t* sfree = &bars[P_FREE + pg];
             const uint32_t tcol = tmem + 64u * pg;
             // this warpgroup's slot in the chain CTA
-            const uint32_t r_sl = tc::mapa(sbase + C_OFF_SL + pg * SZ_CSLOT, 1);
-            const uint32_t r_sc = tc::mapa(sbase + C_OFF_SC + pg * kScalBytes, 1);
+            const uint32_t r_sl = tc::mapa(sbase + C_OFF_SL + pg * SZ_TILES, 1);
+            const uint32_t r_sc0 = tc::mapa(sbase + C_OFF_SC, 1);  // gate-factor ring
             const uint32_t r_tpf = tc::mapa(smem_u32(&bars[C_TPF + pg]), 1);
             const uint32_t idS = tc::idesc_bf16(128, 64, 0, 0);
             auto issue_load = [&](int c) {
@@ -500,25 +499,38 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 loads = 1;
             }
             int n = 0;
-            for (int c = pg; c < nch; c += NPREP, ++n) {
+            // g and beta of a chunk's 64 tokens (thread pt < 64 holds token pt), fetched
+            // one job ahead so their latency overlaps the previous chunk's work
+            auto load_gb = [&](int c, float& gv, float& bv) {
                 const int64_t t0 = cs + (int64_t)C * c;
-                const int len = (int)((ce - t0) < C ? (ce - t0) : C);
-                float gv = 0.f, bv = 0.f;
-                if (pt < len) {
+                gv = 0.f;
+                bv = 0.f;
+                if (c < nch && pt < 64 && t0 + pt < ce) {
                     gv = p.g[(t0 + pt) * H + head];
                     bv = p.beta[(t0 + pt) * H + head];
                 }
+            };
+            float gv_next, bv_next;
+            load_gb(pg, gv_next, bv_next);
+            for (int c = pg; c < nch; c += NPREP, ++n) {
+                const float gv = gv_next, bv = bv_next;
+                load_gb(c + NPREP, gv_next, bv_next);
                 wait(full, n & 1, abort_flag);
-                if (pt == 0) {
+                __syncwarp();
+                if (pw == 0) {
+                    // S_kk = [K; Q] K^T, issued by one elected lane of warp 0
                     tc::tc_after_sync();
-                    const uint32_t lk = tc::desc_lo(kq, 16);
-                    tc::mma_ss<0>(tcol, tc::desc(lk), tc::desc(lk), idS);
+                    if (tc::elect_one()) {
+                        const uint32_t lk = tc::desc_lo(kq, 16);
+                        tc::mma_ss<0>(tcol, tc::desc(lk), tc::desc(lk), idS);
 #pragma unroll
-                    for (int kk = 1; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 2;  // 16-byte units
-                        tc::mma_ss<1>(tcol, tc::desc(lk + off), tc::desc(lk + off), idS);
+                        for (int kk = 1; kk < 8; ++kk) {
+                            const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 2;  // 16-byte units
+                            tc::mma_ss<1>(tcol, tc::desc(lk + off), tc::desc(lk + off), idS);
+                        }
+                        tc::mma_commit(mS);
                     }
-                    tc::mma_commit(mS);
+                    __syncwarp();
                 }
                 // in-chunk inclusive cumsum of g (log2 units) on warps 0-1
                 float x = gv * kLog2e;
@@ -628,9 +640,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 if (pt == 0) {
                     // ship the image once the chain has released the slot
                     if (n >= 1) wait(sfree, (n - 1) & 1, abort_flag, true);
-                    tc::bulk_s2cluster(r_sl + CS_WT, im + SL_TP, 8192, r_tpf);
-                    tc::bulk_s2cluster(r_sl + CS_TB, im + SL_TB, 16384, r_tpf);
-                    tc::bulk_s2cluster(r_sc, cst_u32, kScalBytes, r_tpf);
+                    tc::bulk_s2cluster(r_sl, im, SZ_TILES, r_tpf);
+                    tc::bulk_s2cluster(r_sc0 + (uint32_t)(c % NFAC) * kScalBytes, cst_u32, kScalBytes,
+                                       r_tpf);
                     tc::bulk_commit();
                 }
             }
@@ -656,7 +668,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
         auto kbuf = [&](int c) { return sbase + C_OFF_K + (uint32_t)(c % NKB) * SZ_T; };
         auto vbuf = [&](int c) { return sbase + C_OFF_V + (uint32_t)(c % NVB) * SZ_T; };
         auto qbuf = [&](int c) { return sbase + C_OFF_Q + (uint32_t)(c % NQB) * SZ_T; };
-        auto slot = [&](int c) { return sbase + C_OFF_SL + (uint32_t)(c % NPREP) * SZ_CSLOT; };
+        auto slot = [&](int c) { return sbase + C_OFF_SL + (uint32_t)(c % NPREP) * SZ_TILES; };
+        const uint32_t wt = sbase + C_OFF_WT;
+        const uint32_t ostg = sbase + C_OFF_OUT;
         if (warp == W_LOAD) {
             if (lane == 0) {
                 // loader: K, V and Q tiles as their buffers fall free, and the slots
@@ -675,6 +689,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 uint32_t idle = 0;
                 while (!*abort_flag) {
                     bool prog = false;
+                    if (ns + NPREP < nch && mbar_test(&bars[C_SLOTDONE + ns % NPREP], (ns / NPREP) & 1)) {
+                        // re-arm the slot's barrier for its next image, then hand it back
+                        const int j = ns % NPREP;
+                        tc::mbar_arrive_expect_tx(&bars[C_TPF + j], kImgTx);
+                        tc::mbar_arrive_cluster(r_free0 + 8 * j);
+                        ++ns;
+                        prog = true;
+                    }
                     if (nk < nch && (nk < NKB || mbar_test(&bars[C_KFREE + nk % NKB], ((nk / NKB) - 1) & 1))) {
                         load(&p.tm_k, kbuf(nk), &bars[C_KF + nk % NKB], nk);
                         ++nk;
@@ -688,14 +710,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     if (nq < nch && (nq < NQB || mbar_test(&bars[C_QFREE + nq % NQB], ((nq / NQB) - 1) & 1))) {
                         load(&p.tm_q, qbuf(nq), &bars[C_QF + nq % NQB], nq);
                         ++nq;
-                        prog = true;
-                    }
-                    if (ns + NPREP < nch && mbar_test(&bars[C_SLOTDONE + ns % NPREP], (ns / NPREP) & 1)) {
-                        // re-arm the slot's barrier for its next image, then hand it back
-                        const int j = ns % NPREP;
-                        tc::mbar_arrive_expect_tx(&bars[C_TPF + j], kImgTx);
-                        tc::mbar_arrive_cluster(r_free0 + 8 * j);
-                        ++ns;
                         prog = true;
                     }
                     if (nk == nch && nv == nch && nq == nch && ns + NPREP >= nch) break;
@@ -732,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             auto issue_wt_mmas = [&](int c) {  // W^T(c) = K^T T'^T  (A = K tile MN-major, B = T' K-major)
                 tc::tc_after_sync();
                 if (tc::elect_one()) {
-                    const uint32_t la = lo(kbuf(c), 8192), lb = lo(slot(c) + CS_WT, 16);
+                    const uint32_t la = lo(kbuf(c), 8192), lb = lo(slot(c) + SL_TP, 16);
                     tc::mma_ss<0>(tmem + C_COL_WT, tc::desc(la), tc::desc(lb), idWT);
 #pragma unroll
                     for (int kk = 1; kk < 4; ++kk)
@@ -752,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 __syncwarp();
                 tc::tc_after_sync();
                 if (tc::elect_one()) {
-                    const uint32_t la = lo(vbuf(c), 8192), lb = lo(slot(c) + CS_TB, 16);
+                    const uint32_t la = lo(vbuf(c), 8192), lb = lo(slot(c) + SL_TB, 16);
                     tc::mma_ss<0>(tmem + C_COL_U, tc::desc(la), tc::desc(lb), idU0);
 #pragma unroll
                     for (int kk = 1; kk < 4; ++kk)
@@ -770,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 tc::tc_after_sync();
                 if (tc::elect_one()) {
                     // Ut^T = V^T Tb^T - S W^T
-                    const uint32_t lwt = lo(slot(c) + CS_WT, 8192);
+                    const uint32_t lwt = lo(wt, 8192);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         tc::mma_ts<1>(tmem + C_COL_U, tmem + C_COL_SB + 8 * kk, tc::desc(lwt + 128 * kk), idUt);
@@ -813,12 +827,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     tc::mma_commit(mD);
                     tc::mma_commit(&bars[C_KFREE + c % NKB]);
                     // Ut^T P^T
-                    const uint32_t lp = lo(slot(c) + CS_P, 16);
+                    const uint32_t lp = lo(slot(c) + SL_P, 16);
                     tc::mma_ts<0>(tmem + C_COL_O2, tmem + C_COL_UB, tc::desc(lp), idUP);
 #pragma unroll
                     for (int kk = 1; kk < 4; ++kk)
                         tc::mma_ts<1>(tmem + C_COL_O2, tmem + C_COL_UB + 8 * kk, tc::desc(lp + 2 * kk), idUP);
                     tc::mma_commit(mO);
+                    tc::mma_commit(&bars[C_SLOTDONE + c % NPREP]);  // the slot's tiles are spent
                 }
                 if (c + 1 < nch) {
                     if (!early) issue_wt(c + 1);
@@ -834,22 +849,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
         } else if (warp == W_STORE) {
             if (lane == 0) {
                 // output store warp: sends each full chunk's staged fp32 output out with
-                // four TMA stores (one per value quarter) and frees the slot once the
+                // four TMA stores (one per value quarter) and frees the stage once the
                 // stores have read it; ragged or bf16 chunks were stored directly
                 tc::prefetch_tmap(&p.tm_o);
                 for (int c = 0; c < nch; ++c) {
-                    const int j = c % NPREP;
-                    wait(&bars[C_OUTRDY + j], (c / NPREP) & 1, abort_flag);
+                    wait(&bars[C_OUTRDY], c & 1, abort_flag);
                     const int64_t t0 = cs + (int64_t)C * c;
                     if (!OBF16 && ce - t0 >= C && !*abort_flag) {
 #pragma unroll
                         for (int qq = 0; qq < 4; ++qq)
-                            tc::tma_store_2d(&p.tm_o, slot(c) + (uint32_t)qq * 8192u, head * VD + 32 * qq,
+                            tc::tma_store_2d(&p.tm_o, ostg + (uint32_t)qq * 8192u, head * VD + 32 * qq,
                                              (int)t0);
                         tc::bulk_commit();
                         tc::bulk_wait_read0();
                     }
-                    tc::mbar_arrive(&bars[C_SLOTDONE + j]);
+                    tc::mbar_arrive(&bars[C_STGFREE]);
                 }
                 tc::bulk_wait0();  // the output is in global memory before the CTA leaves
             }
@@ -871,9 +885,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 for (int jj = 0; jj < 32; ++jj) S[jj] = 0.f;
             }
             // W^T (lane = key 32q + lane) tokens 16wg.. -> bf16 row of the MN-major B tile
-            // (into the slot's first 16 KB: the W^T product has read T' there)
-            auto conv_wt = [&](int c) {
-                const uint32_t wt = slot(c) + CS_WT;
+            // (Ut^T of the previous chunk has read the buffer)
+            auto conv_wt = [&]() {
                 float x[16];
                 tc::tmem_ld16(tmem + lane_base + C_COL_WT + 16u * wg, x);
                 tc::tmem_wait_ld();
@@ -896,12 +909,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             if (nch > 0) {
                 wait(mW, 0, abort_flag);
                 tc::tc_after_sync();
-                conv_wt(0);
+                conv_wt();
                 store_sb();
             }
             for (int c = 0; c < nch; ++c) {
                 const int j = c % NPREP;
-                const ChainScal* sc = reinterpret_cast<const ChainScal*>(base + C_OFF_SC) + j;
+                const ChainScal* sc = reinterpret_cast<const ChainScal*>(base + C_OFF_SC) + (c % NFAC);
                 wait(&bars[C_TPF + j], (c / NPREP) & 1, abort_flag, true);
                 wait(mA, c & 1, abort_flag);
                 tc::tc_after_sync();
@@ -925,16 +938,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(s2);
                 }
-                if (c + 1 < nch) {
-                    // next chunk's W^T (Ut^T of this chunk has read the tile)
-                    wait(mW, (c + 1) & 1, abort_flag);
-                    tc::tc_after_sync();
-                    conv_wt(c + 1);
-                }
                 wait(mD, c & 1, abort_flag);
                 tc::tc_after_sync();
                 {
-                    // S <- 2^G2_L S + dS, and its bf16 copy for the next chunk
+                    // S <- 2^G2_L S + dS
                     const float e = sc->eGL;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -945,7 +952,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                         for (int jj = 0; jj < 16; ++jj) S[16 * h + jj] = fmaf(e, S[16 * h + jj], d[jj]);
                     }
                 }
-                if (c + 1 < nch) store_sb();  // S Q^T and Ut^T of this chunk completed before dS
+                if (c + 1 < nch) {
+                    // next chunk's W^T (Ut^T of this chunk has read the tile), then the bf16
+                    // copy of S (S Q^T and Ut^T of this chunk completed before dS)
+                    wait(mW, (c + 1) & 1, abort_flag);
+                    tc::tc_after_sync();
+                    conv_wt();
+                    store_sb();
+                }
                 {
                     // o_t = scale gam_t (S Q^T)[vr][t] + (Ut^T P'^T)[vr][t] (P' = scale P) for
                     // this warpgroup's 16 tokens, staged in the spent slot for the store warp
@@ -963,9 +977,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                     if (lane == 0) tc::mbar_arrive(ofree);
                     float gm[16];
                     lds16(smem_u32(sc->gam + 16 * wg), gm);
+                    // one output in flight: the previous chunk's has left the stage
+                    if (c >= 1) wait(&bars[C_STGFREE], (c - 1) & 1, abort_flag);
                     if (!OBF16 && len == C) {
                         // 128-byte swizzle: 16-byte chunk lane/4 of row t sits at (lane/4) ^ (t & 7)
-                        const uint32_t a0 = slot(c) + (uint32_t)q * 8192u + 4u * (uint32_t)(lane & 3);
+                        const uint32_t a0 = ostg + (uint32_t)q * 8192u + 4u * (uint32_t)(lane & 3);
                         const uint32_t ch = (uint32_t)(lane >> 2);
                         uint32_t ak[8];
 #pragma unroll
@@ -989,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                         }
                     }
                     __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&bars[C_OUTRDY + j]);  // gate factors read, output staged
+                    if (lane == 0) tc::mbar_arrive(&bars[C_OUTRDY]);  // output staged (or stored)
                 }
             }
             if (p.hT) {
