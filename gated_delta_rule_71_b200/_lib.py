@@ -39,6 +39,7 @@ SIGNATURES = {
     "gdn_conv1d_fwd": (I32, [P, I32, P, P, I32, P, I32, I32, I64, I32, P, P, I32, P, P]),
     "gdn_conv1d_update": (I32, [P, I32, P, P, I32, P, P, I32, I32, I32, I32, P, P]),
     "gdn_device_status": (I32, [P]),
+    "gdn_get_device_status": (I32, [P]),
     "gdn_selftest_wait_timeout": (I32, [U32, P]),
 }
 

@@ -2,6 +2,7 @@
 // argument checks, kernel selection and launches.  One translation unit holds
 // every kernel so that the device status word is a single symbol.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <cstring>
@@ -562,6 +563,8 @@ gdn_status gdn_device_status(void* stream) {
     return (gdn_status)word;
 }
 
+gdn_status gdn_get_device_status(void* stream) { return gdn_device_status(stream); }
+
 }  // extern "C"
 
 namespace gdn {
@@ -589,30 +592,63 @@ extern "C" gdn_status gdn_selftest_wait_timeout(unsigned polls, void* stream) {
 // schedule of a packed batch -- lives in this fixed device array instead of a
 // caller-provided workspace.  Host code must not hand the array's name to a
 // kernel: on the host it is only a stand-in symbol, so its device address is
-// looked up once per device with cudaGetSymbolAddress and cached.
+// looked up with cudaGetSymbolAddress once per CUDA context (the array has one
+// instance per context that loads this module) and cached under that context.
 static __device__ __align__(256) int32_t g_noalloc_schedule[GDN_NOALLOC_MAX_SEQS];
 
 namespace {
-constexpr int kNoAllocMaxDevices = 64;
+constexpr int kNoAllocMaxContexts = 64;
 std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+CUcontext g_noalloc_ctx[kNoAllocMaxContexts] = {};
+void* g_noalloc_addr[kNoAllocMaxContexts] = {};
+int g_noalloc_used = 0;
 
-// Device address of g_noalloc_schedule on the current device; looked up on the
-// first call for that device (this is why that first call must not be made
+// The calling thread's current CUDA context (the device's primary context once
+// the runtime has initialised it), through the driver entry point the runtime
+// exposes, so the library needs no link against the driver library.
+gdn_status current_context(CUcontext* out) {
+    static PFN_cuCtxGetCurrent_v4000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    }();
+    if (!fn) return GDN_ERR_CUDA;
+    *out = nullptr;
+    if (fn(out) != CUDA_SUCCESS) return GDN_ERR_CUDA;
+    if (!*out) {
+        // nothing current on this thread yet: let the runtime make its context current
+        gdn_status s = cuda_check(cudaFree(nullptr));
+        if (s != GDN_OK) return s;
+        if (fn(out) != CUDA_SUCCESS || !*out) return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
+}
+
+// Device address of g_noalloc_schedule in the current context; looked up on the
+// first call in that context (this is why that first call must not be made
 // while a stream is being captured).
 gdn_status noalloc_schedule_addr(void** out) {
-    int dev = 0;
-    gdn_status s = cuda_check(cudaGetDevice(&dev));
+    CUcontext ctx = nullptr;
+    gdn_status s = current_context(&ctx);
     if (s != GDN_OK) return s;
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return GDN_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_addr[dev]) {
-        void* p = nullptr;
-        s = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_schedule));
-        if (s != GDN_OK) return s;
-        g_noalloc_addr[dev] = p;
+    for (int i = 0; i < g_noalloc_used; ++i)
+        if (g_noalloc_ctx[i] == ctx) {
+            *out = g_noalloc_addr[i];
+            return GDN_OK;
+        }
+    void* p = nullptr;
+    s = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_schedule));
+    if (s != GDN_OK) return s;
+    if (g_noalloc_used < kNoAllocMaxContexts) {
+        g_noalloc_ctx[g_noalloc_used] = ctx;
+        g_noalloc_addr[g_noalloc_used] = p;
+        ++g_noalloc_used;
     }
-    *out = g_noalloc_addr[dev];
+    *out = p;
     return GDN_OK;
 }
 }  // namespace
@@ -628,9 +664,11 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const 
     size_t ws_bytes = 0;
     if (cu_seqlens) {
         if (n_seq > GDN_NOALLOC_MAX_SEQS) return GDN_ERR_TOO_LARGE;
-        if (n_seq > 1) {
-            // every entry the schedule kernel later reads it first writes, so the
-            // array needs no clearing between calls
+        if (n_seq >= 1) {
+            // gdn_chunk_fwd wants a schedule buffer for every packed batch (even one
+            // of a single sequence, whose schedule it does not build); every entry
+            // the schedule kernel later reads it first writes, so the array needs
+            // no clearing between calls
             gdn_status s = noalloc_schedule_addr(&ws);
             if (s != GDN_OK) return s;
             ws_bytes = sizeof(g_noalloc_schedule);

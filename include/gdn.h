@@ -118,14 +118,15 @@ size_t gdn_chunk_fwd_workspace_size(int n_seq, int64_t T_total, int H, int K, in
  *   hT      : fp32 [n_seq, H, K, V] final states, written; NULL to skip.
  *   workspace / ws_bytes : device scratch of gdn_chunk_fwd_workspace_size(...)
  *             bytes.  Its contents on entry do not matter.  A packed batch
- *             needs at least its schedule (4 * n_seq bytes, rounded up to 256);
- *             a dense batch may pass NULL.  With less than the full size the
- *             bf16 K = V = 128 path runs as one cluster of two CTAs per
- *             (sequence, head); with the full size, a dense batch whose
- *             n_seq * H chains fit in two thirds of the SMs runs as one
- *             cooperative launch (chains on n_seq * H CTAs, the WY prep of
- *             every (chunk, head) on the other SMs), which is faster.
+ *             needs its longest-first schedule (4 * n_seq bytes, rounded up
+ *             to 256), a single sequence included; a dense batch needs none
+ *             and may pass NULL.  The bf16 K = V = 128 path runs as one
+ *             cluster of two CTAs per (sequence, head): the WY prep of every
+ *             chunk on one, the inter-chunk recurrence and the output on the
+ *             other.
  *   flags   : GDN_FLAG_* bits; 0 selects the fastest kernel for the dtype.
+ *             (An addition to the call list the method's API describes, which
+ *             has no flags argument: pass 0 for exactly that call.)
  * Supported: K, V in {32, 64, 128}.  bf16 q/k/v run on the tcgen05 tensor-core
  * kernel (bf16 operands, fp32 accumulation and fp32 state) when K = V = 128;
  * otherwise, and for fp32 q/k/v, an fp32-FMA kernel that keeps every product
@@ -255,9 +256,11 @@ gdn_status gdp_prefill(const void* x, int64_t x_n_stride, const void* ba, int64_
  * library keeps until the process exits.  It calls no allocator at all.
  *  - cu_seqlens != NULL with n_seq > GDN_NOALLOC_MAX_SEQS returns
  *    GDN_ERR_TOO_LARGE and launches nothing (dense batches have no limit).
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before capturing a stream into a CUDA graph.
+ *  - The first call in each CUDA context (the primary context of each device,
+ *    for runtime-API callers) looks up the array's device address
+ *    (cudaGetSymbolAddress, with that context current) and caches it under the
+ *    context; make that first call before capturing a stream into a CUDA graph.
+ *  - A packed batch of any size, one sequence included, uses the array.
  *  - All calls share the one array, and every call overwrites the entries it
  *    uses before reading them, so nothing carries over between calls; but two
  *    calls that run on the GPU at the same time (different streams, or
@@ -346,6 +349,10 @@ gdn_status gdn_accumulate_f32(float* y, const float* x, int64_t n, void* stream)
  * stream.  Returns GDN_OK when nothing was recorded.
  */
 gdn_status gdn_device_status(void* stream);
+
+/* gdn_get_device_status -- the same call under the name of the method's API
+ * call list (reads and clears the device status word; synchronises). */
+gdn_status gdn_get_device_status(void* stream);
 
 /*
  * gdn_selftest_wait_timeout -- launches one block that waits on an mbarrier

@@ -32,6 +32,16 @@ def test_every_declared_symbol_is_exported():
     assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
 
 
+def test_the_method_call_list_is_exported():
+    # the entry points of the method's API call list, by their names there
+    lib = ctypes.CDLL(LIB)
+    for n in ("gdn_gate_prep", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd",
+              "gdp_decode_prepare", "gdp_decode_step", "gdn_get_device_status",
+              "gdn_status_string"):
+        assert hasattr(lib, n), n
+        assert n in _declared(), n
+
+
 def test_status_strings():
     lib = _lib.load()
     for s in range(5):
