@@ -13,7 +13,7 @@ import torch
 import gated_delta_rule_71_b200 as gdn
 import oracle
 from gated_delta_rule_71_b200 import inputs as I
-from tests._util import TOL_BF16, TOL_F32, oracle_sampled, relerr, to_dev, ulp_dist
+from tests._util import TOL_BF16, TOL_F32, relerr, to_dev, ulp_dist
 
 pytestmark = pytest.mark.gpu
 
@@ -185,18 +185,69 @@ def test_tensor_core_path_matches_oracle(cuda_device, B, T, H, h0):
 
 # ------------------------------------------------- full-size workloads, sampled
 
-@pytest.mark.parametrize("w,pairs", [
-    (I.BF16_B4_T4096, [(0, 0), (1, 7), (2, 11), (3, 15)]),
-    (I.VARLEN_8x32768, [(0, 0), (3, 17), (5, 31), (7, 8)]),
-    (I.LONG_T131072, [(0, 0), (0, 21)]),
+def _elem_err(x, ref):
+    """Elementwise relative error |x - y| / max(|y|, 1e-6 max|y|): its maximum and
+    99.9th percentile (the floor keeps elements that are zero to within rounding
+    from dividing by nothing)."""
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.maximum(np.abs(ref), 1e-6 * np.abs(ref).max())
+    e = np.abs(x - ref) / den
+    return float(e.max()), float(np.quantile(e, 0.999))
+
+
+def _report(case, **kw):
+    import json
+    import os
+    path = os.environ.get("GDN_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(case=case, **kw)) + "\n")
+
+
+def _heads(inp, beta, g, heads):
+    """The inputs restricted to a subset of heads (all sequences kept)."""
+    sel = lambda t: t[:, :, heads].contiguous()
+    h0 = None if inp["h0"] is None else inp["h0"][:, heads].contiguous()
+    return (sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), sel(g), sel(beta), h0)
+
+
+# c1: every batch entry x 4 heads; c2: every packed sequence x 4 heads;
+# c3: the one sequence x 8 heads.  The oracle runs the selected chains on all
+# host cores at once.
+@pytest.mark.parametrize("w,heads", [
+    (I.BF16_B4_T4096, [0, 5, 10, 15]),
+    (I.VARLEN_8x32768, [0, 9, 17, 31]),
+    (I.LONG_T131072, [0, 3, 7, 12, 16, 21, 26, 31]),
 ])
-def test_full_size_sampled(cuda_device, w, pairs):
+def test_full_size_sampled(cuda_device, w, heads):
     inp = I.chunk_inputs(w)
-    o, hT, beta, g = _run(inp, cuda_device)
+    d = to_dev(inp, cuda_device)
+    beta, g = gdn.gate_prep(d["a"], d["b"], d["A_log"], d["dt_bias"])
+    o, hT = gdn.chunk_fwd(d["q"], d["k"], d["v"], g, beta, h0=d["h0"], cu_seqlens=d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
     assert torch.isfinite(o).all() and torch.isfinite(hT).all()
-    for (s, h), (ro, rh, (b, r0, r1)) in oracle_sampled(inp, beta, g, pairs).items():
-        assert relerr(o[b, r0:r1, h], ro) <= TOL_BF16, (s, h)
-        assert relerr(hT[s, h], rh) <= TOL_BF16, (s, h)
+    idx = torch.tensor(heads, device=cuda_device)
+    o_s = o.index_select(2, idx).cpu()
+    h_s = hT.index_select(1, idx).cpu()
+    del o, hT, d
+    q, k, v, gs, bs, h0 = _heads(inp, beta.cpu(), g.cpu(), heads)
+    ro, rh = oracle.gdn_fwd(q, k, v, gs, bs, h0=h0, cu_seqlens=inp["cu_seqlens"])
+    n_seq = rh.shape[0]
+    cu = inp["cu_seqlens"]
+    worst_o = worst_h = 0.0
+    for s in range(n_seq):
+        b, r0, r1 = (s, 0, o_s.shape[1]) if cu is None else (0, int(cu[s]), int(cu[s + 1]))
+        for j, h in enumerate(heads):
+            eo = relerr(o_s[b, r0:r1, j], ro[b, r0:r1, j]) if r1 > r0 else 0.0
+            eh = relerr(h_s[s, j], rh[s, j])
+            assert eo <= TOL_BF16 and eh <= TOL_BF16, (s, h, eo, eh)
+            worst_o, worst_h = max(worst_o, eo), max(worst_h, eh)
+    eo_max, eo_q = _elem_err(o_s.numpy(), ro)
+    eh_max, eh_q = _elem_err(h_s.numpy(), rh)
+    _report(w.name, chains=n_seq * len(heads), normwise_o=worst_o, normwise_hT=worst_h,
+            elem_o_max=eo_max, elem_o_p999=eo_q, elem_hT_max=eh_max, elem_hT_p999=eh_q)
 
 
 # ------------------------------------------------------------------ decode
