@@ -388,6 +388,38 @@ def run_ours(args):
     dby, dfl = decode_algorithmic(dw.n, *dargs)
     dach = dby / (dec_ms * 1e-3) / 1e9
 
+    # --- the decode token of a layer in one launch (conv update + decode step) against
+    # the same two launches apart, on the decode workload with a W=4 SiLU convolution
+    Cd = dw.M * dw.H * dw.P + dw.M * dw.G * dw.N + dw.G * dw.N
+    lcv = {k: v.to(dev) for k, v in I.conv_decode_inputs(dw.n, Cd, 4, dw.n, seed=1011).items()}
+    lx = dd["x"].reshape(dw.n, Cd)
+    lba = dd["ba"].reshape(dw.n, -1)
+    lws = torch.zeros(gdn.gdp_decode_layer_step_workspace_size(dw.n, dw.G), dtype=torch.uint8,
+                      device=dev)
+    ly = torch.empty_like(lx)
+
+    def layer_fused():
+        gdn.gdp_decode_layer_step(lx, lba, lcv["w"], lcv["conv_state"], dd["A_log"], dd["dt_bias"],
+                                  dd["state"], *dargs, conv_bias=lcv["bias"], out=od, workspace=lws)
+
+    def layer_two():
+        gdn.conv1d_update(lx, lcv["w"], lcv["conv_state"], lcv["bias"], activation=True, out=ly)
+        gdn.gdp_decode_step(ly, lba, dd["A_log"], dd["dt_bias"], dd["state"], *dargs, out=od)
+
+    lay_ms = {}
+    for nm, fn in (("fused", layer_fused), ("two_launches", layer_two)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        d0.record(stream)
+        for _ in range(n_dec):
+            fn()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        lay_ms[nm] = max_over_ranks(d0.elapsed_time(d1), world, dev) / n_dec
+    lay_by = dby + dw.n * Cd * 3 * 2 * 2 + Cd * 4 * 4 + Cd * 4
+    lay_ach = lay_by / (lay_ms["fused"] * 1e-3) / 1e9
+
     # --- short convolution (ZzCompute item 1) over the layer's q/k/v channels, and its
     # one-token update at the decode row width
     cw = I.CONV_B4_T4096
@@ -483,6 +515,16 @@ def run_ours(args):
                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                     "frac": round(dach / peaks["hbm_gbs"], 4),
                                     "algorithmic_bytes": dby}},
+            "decode_layer": {"workload": dw.name + " + conv W4 SiLU", "metric": "requests/s",
+                             "value": dw.n * world / (lay_ms["fused"] * 1e-3),
+                             "ms_per_step": lay_ms["fused"],
+                             "two_launches_ms": lay_ms["two_launches"],
+                             "path": "gdp_decode_layer_step (one launch) vs gdn_conv1d_update + "
+                                     "gdp_decode_step",
+                             "roofline": {"bound": "hbm", "achieved": round(lay_ach, 1),
+                                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                          "frac": round(lay_ach / peaks["hbm_gbs"], 4),
+                                          "algorithmic_bytes": lay_by}},
             "conv1d": {"workload": cw.name, "metric": "tokens/s",
                        "value": cw.B * cw.T * world / (conv_ms * 1e-3), "ms_per_step": conv_ms,
                        "roofline": {"bound": "hbm", "achieved": round(conv_ach, 1),

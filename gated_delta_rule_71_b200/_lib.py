@@ -29,6 +29,11 @@ SIGNATURES = {
                               P]),
     "gdp_decode_step_indexed": (I32, [P, I64, P, I64, P, P, I32, I32, I32, I32, I32, I32, P, P,
                                       I32, P, F32, I32, P]),
+    "gdp_decode_layer_step_workspace_size": (SZ, [I32, I32]),
+    # x, xs, ba, bas, conv_w, conv_bias, W, conv_state, activation, A_log, dt_bias,
+    # n, M, H, G, P, N, state, state_idx, n_slots, o, scale, qk_l2norm, workspace, ws_bytes, stream
+    "gdp_decode_layer_step": (I32, [P, I64, P, I64, P, P, I32, P, I32, P, P, I32, I32, I32, I32, I32,
+                                    I32, P, P, I32, P, F32, I32, P, SZ, P]),
     "gdp_prefill_workspace_size": (SZ, [I32, I64, I32, I32, I32, I32, I32, I32]),
     "gdp_prefill": (I32, [P, I64, P, I64, P, P, P, P, I32, I32, I64, I32, I32, I32, I32, I32,
                           F32, P, I32, P, P, SZ, P]),

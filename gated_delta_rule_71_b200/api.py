@@ -183,6 +183,57 @@ def gdp_decode_step(x, ba, A_log, dt_bias, state, M, H, G, P, N, scale=1.0, qk_l
     return out
 
 
+def gdp_decode_layer_step_workspace_size(n, G):
+    return int(_lib.load().gdp_decode_layer_step_workspace_size(n, G))
+
+
+def gdp_decode_layer_step(x, ba, conv_w, conv_state, A_log, dt_bias, state, M, H, G, P, N,
+                          conv_bias=None, activation=True, scale=1.0, qk_l2norm=True,
+                          state_indices=None, out=None, workspace=None):
+    """One decode token of a layer in one launch: the short-convolution update of
+    the projected rows x [n, C] (bf16, before the convolution; conv_state
+    [n_slots, C, W-1] bf16 updated in place, conv_w [C, W] fp32), then the decode
+    step on the convolved rows.  Arguments otherwise as gdp_decode_step (one slot
+    index names both the conv window and the state).  workspace: uint8 tensor of
+    gdp_decode_layer_step_workspace_size(n, G) bytes, zero before its first use
+    and left zero by every call; None allocates a zeroed one."""
+    dev, n, xs, bas = _decode_common(x, ba, A_log, dt_bias, M, H, G, P, N)
+    C = M * H * P + M * G * N + G * N
+    _need(conv_w, "conv_w", torch.float32, dev)
+    if conv_w.dim() != 2 or conv_w.shape[0] != C:
+        raise ValueError("conv_w must be [C, W] with C = M*H*P + M*G*N + G*N")
+    W = conv_w.shape[1]
+    _need(conv_state, "conv_state", torch.bfloat16, dev)
+    if conv_state.dim() != 3 or tuple(conv_state.shape[1:]) != (C, W - 1):
+        raise ValueError("conv_state must be [n_slots, C, W-1]")
+    if conv_bias is not None:
+        _need(conv_bias, "conv_bias", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    if state.dim() != 4 or tuple(state.shape[1:]) != (H, N, P):
+        raise ValueError("state must be [n_slots, H, N, P]")
+    n_slots = state.shape[0]
+    if conv_state.shape[0] != n_slots:
+        raise ValueError("conv_state and state must have the same number of slots")
+    if state_indices is None:
+        if n_slots < n:
+            raise ValueError("without state_indices, state must have at least n slots")
+    else:
+        _need(state_indices, "state_indices", torch.int32, dev)
+        if tuple(state_indices.shape) != (n,):
+            raise ValueError("state_indices must be int32 [n]")
+    if out is None:
+        out = torch.empty((n, H, P), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    ws_need = gdp_decode_layer_step_workspace_size(n, G)
+    if workspace is None:
+        workspace = torch.zeros(max(ws_need, 1), dtype=torch.uint8, device=dev)
+    _lib.call("gdp_decode_layer_step", _ptr(x), xs, _ptr(ba), bas, _ptr(conv_w), _ptr(conv_bias),
+              W, _ptr(conv_state), int(bool(activation)), _ptr(A_log), _ptr(dt_bias), n, M, H, G,
+              P, N, _ptr(state), _ptr(state_indices), n_slots, _ptr(out), float(scale),
+              int(bool(qk_l2norm)), _ptr(workspace), workspace.numel(), _stream(x))
+    return out
+
+
 def gdp_prefill_workspace_size(n_seq, rows, M, H, P, N, o_dtype=torch.float32, packed=False):
     return int(_lib.load().gdp_prefill_workspace_size(n_seq, rows, M, H, P, N, _DT[o_dtype],
                                                       int(bool(packed))))

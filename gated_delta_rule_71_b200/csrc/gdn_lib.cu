@@ -15,6 +15,7 @@
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
 #include "conv1d.cuh"
+#include "decode_step.cuh"
 
 namespace {
 
@@ -163,6 +164,33 @@ gdn_status conv_upd_t(const gdn::ConvUpdateArgs& a, int W, bool act, bool vec,
     constexpr int NV = gdn::ConvVec<T>::N;
     if (vec) return act ? conv_upd_w<T, NV, true>(a, W, st) : conv_upd_w<T, NV, false>(a, W, st);
     return act ? conv_upd_w<T, 1, true>(a, W, st) : conv_upd_w<T, 1, false>(a, W, st);
+}
+
+// The decode step (FUSED: behind the short-convolution update of its row).
+// 64-column state slabs for P >= 64 (two blocks per (request, head) at P = 128),
+// so four blocks fit per SM and one block's state loads overlap another's
+// arithmetic.
+template <bool FUSED>
+gdn_status launch_decode(const void* x, int64_t xs, const void* ba, int64_t bas,
+                         const float* A_log, const float* dt_bias, int n, int M, int H, int G,
+                         int P, int N, float* state, const int32_t* state_idx, int n_slots,
+                         void* o, float scale, int l2, const gdn::dec::ConvIn& cv,
+                         cudaStream_t st) {
+    using bf = __nv_bfloat16;
+    const int nb = n * H;
+#define GDN_DEC(NN, PP)                                                                          \
+    if (N == NN && P == PP) {                                                                    \
+        constexpr int PB = PP >= 64 ? 64 : PP;                                                   \
+        gdn::dec::step_kernel<NN, PP, PB, FUSED><<<nb * (PP / PB), 256, 0, st>>>(                \
+            (const bf*)x, xs, (const bf*)ba, bas, A_log, dt_bias, M, H, G, state, state_idx,     \
+            n_slots, (bf*)o, scale, l2, cv);                                                     \
+        return launch_check();                                                                   \
+    }
+    GDN_DEC(128, 128) GDN_DEC(128, 64) GDN_DEC(128, 32)
+    GDN_DEC(64, 128) GDN_DEC(64, 64) GDN_DEC(64, 32)
+    GDN_DEC(32, 128) GDN_DEC(32, 64) GDN_DEC(32, 32)
+#undef GDN_DEC
+    return GDN_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -336,23 +364,9 @@ gdn_status gdp_decode_step_indexed(const void* x, int64_t x_n_stride, const void
     using bf = __nv_bfloat16;
     const int nb = n * H;
     cudaStream_t st = as_stream(stream);
-    // 64-column slabs for P >= 64 (two blocks per (request, head) at P = 128): four
-    // blocks fit per SM, so one block's state loads overlap another's arithmetic
-    // (measured 0.787 -> 0.822 of the HBM copy bandwidth at n=256 M=2 H=32 G=16 P=N=128;
-    // 32-column slabs were slower, 0.695)
-#define GDN_DEC(NN, PP)                                                                          \
-    if (N == NN && P == PP) {                                                                    \
-        constexpr int PB = PP >= 64 ? 64 : PP;                                                   \
-        gdn::gdp_step_kernel<NN, PP, PB><<<nb * (PP / PB), 256, 0, st>>>(                         \
-            (const bf*)x, x_n_stride, (const bf*)ba, ba_n_stride, A_log, dt_bias, M, H, G, state, \
-            state_idx, n_slots, (bf*)o, scale, qk_l2norm);                                       \
-        return launch_check();                                                                   \
-    }
-    GDN_DEC(128, 128) GDN_DEC(128, 64) GDN_DEC(128, 32)
-    GDN_DEC(64, 128) GDN_DEC(64, 64) GDN_DEC(64, 32)
-    GDN_DEC(32, 128) GDN_DEC(32, 64) GDN_DEC(32, 32)
-#undef GDN_DEC
-    return GDN_ERR_UNSUPPORTED;
+    return launch_decode<false>(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P, N,
+                                state, state_idx, n_slots, o, scale, qk_l2norm, gdn::dec::ConvIn{},
+                                as_stream(stream));
 }
 
 gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, int64_t ba_n_stride,
@@ -362,6 +376,38 @@ gdn_status gdp_decode_step(const void* x, int64_t x_n_stride, const void* ba, in
     if (n > 0 && !state) return GDN_ERR_INVALID_ARG;
     return gdp_decode_step_indexed(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P,
                                    N, state, nullptr, n, o, scale, qk_l2norm, stream);
+}
+
+size_t gdp_decode_layer_step_workspace_size(int n, int G) {
+    if (n <= 0 || G <= 0) return 0;
+    return ((size_t)n * G * 4 + 255) / 256 * 256;
+}
+
+gdn_status gdp_decode_layer_step(const void* x, int64_t x_n_stride, const void* ba,
+                                 int64_t ba_n_stride, const float* conv_w, const float* conv_bias,
+                                 int W, void* conv_state, int activation, const float* A_log,
+                                 const float* dt_bias, int n, int M, int H, int G, int P, int N,
+                                 float* state, const int32_t* state_idx, int n_slots, void* o,
+                                 float scale, int qk_l2norm, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+    gdn_status s = decode_args_ok(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P, N);
+    if (s != GDN_OK) return s;
+    if (W < 1 || W > 4 || (activation != 0 && activation != 1)) return GDN_ERR_INVALID_ARG;
+    if (n == 0) return GDN_OK;
+    if (!o || !conv_w || (W > 1 && !conv_state) || n_slots < 0 || (!state_idx && n_slots < n))
+        return GDN_ERR_INVALID_ARG;
+    if (n_slots > 0 && (!state || !aligned16(state))) return GDN_ERR_INVALID_ARG;
+    if (state_idx && (reinterpret_cast<uintptr_t>(state_idx) & 3u)) return GDN_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < gdp_decode_layer_step_workspace_size(n, G) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    if (M > gdn::dec::kMaxM) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)n * H * 2 > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    const gdn::dec::ConvIn cv{conv_w, conv_bias, static_cast<__nv_bfloat16*>(conv_state),
+                              static_cast<int32_t*>(workspace), W, activation};
+    return launch_decode<true>(x, x_n_stride, ba, ba_n_stride, A_log, dt_bias, n, M, H, G, P, N,
+                               state, state_idx, n_slots, o, scale, qk_l2norm, cv,
+                               as_stream(stream));
 }
 
 }  // extern "C"

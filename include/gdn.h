@@ -209,6 +209,43 @@ gdn_status gdp_decode_step_indexed(const void* x, int64_t x_n_stride, const void
                                    int qk_l2norm, void* stream);
 
 /*
+ * gdp_decode_layer_step -- one decode token of a Gated Delta Product layer in
+ * one launch: the short-convolution update of the projected row (as
+ * gdn_conv1d_update, bf16, over all M*H*P + M*G*N + G*N channels of x), then
+ * gdp_decode_step_indexed on the convolved row.  Megatron-Core
+ * "core.ssm.ops.gdp.decode_prepare", module description: the short-conv update
+ * runs between the projection and the recurrent kernel, and a -1 slot zeroes
+ * its conv output (so o = 0 and neither state is touched).  The results equal,
+ * bit for bit, gdn_conv1d_update (bf16 output) followed by
+ * gdp_decode_step_indexed, without the convolved row going through memory.
+ *   x          : bf16 [n, *] rows BEFORE the short convolution, row stride
+ *                x_n_stride elements, each [value | key | query] as in
+ *                gdp_decode_prepare.  ba, A_log, dt_bias as gdp_decode_step.
+ *   conv_w     : fp32 [C, W], C = M*H*P + M*G*N + G*N;  conv_bias fp32 [C] or
+ *                NULL;  W in 1..4;  activation 1 = SiLU, 0 = none.
+ *   conv_state : bf16 [n_slots, C, W-1], in place (NULL allowed when W == 1).
+ *   state, state_idx, n_slots, o, scale, qk_l2norm : as gdp_decode_step_indexed;
+ *                one slot index names both the conv window and the state.
+ *   workspace  : >= gdp_decode_layer_step_workspace_size(n, G) bytes, 4-byte
+ *                aligned, ZERO before the first call (cudaMemset); every call
+ *                leaves it zero.  It counts, per (request, group), the blocks
+ *                that have read the group's key and query windows, so that the
+ *                last of them shifts those windows after all have read them.
+ *                Calls sharing one workspace must not run concurrently.
+ * Errors: as gdp_decode_step_indexed; INVALID_ARG also for W outside 1..4,
+ * activation not 0/1, NULL conv_w (or conv_state with W > 1), a missing or
+ * short workspace.
+ */
+size_t gdp_decode_layer_step_workspace_size(int n, int G);
+gdn_status gdp_decode_layer_step(const void* x, int64_t x_n_stride, const void* ba,
+                                 int64_t ba_n_stride, const float* conv_w, const float* conv_bias,
+                                 int W, void* conv_state, int activation, const float* A_log,
+                                 const float* dt_bias, int n, int M, int H, int G, int P, int N,
+                                 float* state, const int32_t* state_idx, int n_slots, void* o,
+                                 float scale, int qk_l2norm, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
+/*
  * gdp_prefill -- the Gated Delta Product over a whole prompt: every token row
  * carries the decode layout (x row [value: M*H*P | key: M*G*N | query: G*N],
  * ba row [b: M*H | a: H], as in gdp_decode_prepare), and the rule runs over the
