@@ -1,9 +1,8 @@
-// gates_decode.cuh -- gate preparation and the Gated Delta Product decode step.
+// gates_decode.cuh -- gate preparation, the decode prepare and the CP helpers.
 //
 // Gates: Megatron-Core "core.ssm.ops.gdp.decode_prepare", module description and
 // the `softplus` entry.  Decode layout: the `gdp_decode_prepare` function entry
 // (post-conv row [value | key | query], ba row [b | a], outputs [n, M, H, *]).
-// The state update is the gated delta rule run over the M Householder copies.
 #pragma once
 
 #include "common.cuh"
@@ -75,173 +74,7 @@ __global__ void __launch_bounds__(256) gdp_prepare_kernel(
     }
 }
 
-// ---------------------------------------------------------------- decode step
-// One block (8 warps) per (request, head).  The request's state sits in slot
-// state_idx[r] of the state pool (slot r when state_idx is NULL); a negative
-// slot is a padding request: o = 0 and its state is neither read nor written
-// (Megatron-Core "core.ssm.ops.gdp.decode_prepare", module description: the
-// batch is padded upstream with -1 slots).  A slot >= n_slots is handled the
-// same way and records GDN_ERR_INVALID_ARG in the device status word.  The
-// value columns of the state never interact, so a (request, head) is split
-// over P / PB blocks of PB columns each (smaller blocks: more of them resident
-// per SM to overlap one block's loads with another's arithmetic).  The block's
-// fp32 state slab [N, PB] lives in registers: warp w owns key rows
-// [w*N/8, (w+1)*N/8), lane l owns columns [l*PB/32, (l+1)*PB/32), so every row
-// is read and written as one coalesced warp access.  Column reductions over the key
-// axis go through shared memory.  The state is read once and written once:
-// the kernel is HBM-bound on 2*N*P*4 bytes per (request, head).
-constexpr int kDecWarps = 8;
-constexpr int kDecMaxM = 8;
-
-template <int N, int P, int PB>
-__global__ void __launch_bounds__(256, (PB <= 64 ? 4 : 2)) gdp_step_kernel(
-    const __nv_bfloat16* __restrict__ x, int64_t xs, const __nv_bfloat16* __restrict__ ba,
-    int64_t bas, const float* __restrict__ A_log, const float* __restrict__ dt_bias, int M, int H,
-    int G, float* __restrict__ state, const int32_t* __restrict__ state_idx, int n_slots,
-    __nv_bfloat16* __restrict__ o, float scale, int l2) {
-    constexpr int RPW = N / kDecWarps;  // rows per warp
-    constexpr int CPL = PB / 32;        // columns per lane
-    constexpr int NPART = P / PB;
-    __shared__ float kv[kDecMaxM][N];
-    __shared__ float vv[kDecMaxM][PB];
-    __shared__ float qv[N];
-    __shared__ float red[kDecWarps][PB];
-    __shared__ float uu[PB];
-    __shared__ float gate_b[kDecMaxM];
-    __shared__ float gate_e;
-
-    const int rh = blockIdx.x / NPART;  // request * H + head
-    const int p0 = (blockIdx.x - rh * NPART) * PB;  // first value column of this block
-    const int r = rh / H, h = rh - r * H;
-    const int hpg = H / G, grp = h / hpg;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const __nv_bfloat16* xr = x + (int64_t)r * xs;
-    const __nv_bfloat16* br = ba + (int64_t)r * bas;
-    const int64_t kbase = (int64_t)M * H * P, qbase = kbase + (int64_t)M * G * N;
-    const int slot = state_idx ? state_idx[r] : r;
-    if (slot < 0 || slot >= n_slots) {  // padding (uniform across the block)
-        if (slot >= n_slots && threadIdx.x == 0) record_status(GDN_ERR_INVALID_ARG);
-        if (threadIdx.x < PB) o[(int64_t)rh * P + p0 + threadIdx.x] = __float2bfloat16_rn(0.f);
-        return;
-    }
-
-    // 1. issue the state loads first (the only large traffic)
-    float* st = state + ((int64_t)slot * H + h) * N * P + p0;
-    float s[RPW][CPL];
-#pragma unroll
-    for (int rr = 0; rr < RPW; ++rr) {
-        const float* src = st + (int64_t)(warp * RPW + rr) * P + lane * CPL;
-        if constexpr (CPL == 4) {
-            float4 t = *reinterpret_cast<const float4*>(src);
-            s[rr][0] = t.x; s[rr][1] = t.y; s[rr][2] = t.z; s[rr][3] = t.w;
-        } else if constexpr (CPL == 2) {
-            float2 t = *reinterpret_cast<const float2*>(src);
-            s[rr][0] = t.x; s[rr][1] = t.y;
-        } else {
-            s[rr][0] = src[0];
-        }
-    }
-
-    // 2. split / GQA-expand / normalise the M copies and the query into smem
-    for (int m = warp; m <= M; m += kDecWarps) {
-        const __nv_bfloat16* src = (m < M) ? xr + kbase + ((int64_t)m * G + grp) * N
-                                           : xr + qbase + (int64_t)grp * N;
-        float e[N / 32];
-        float ss = 0.f;
-#pragma unroll
-        for (int i = 0; i < N / 32; ++i) {
-            e[i] = __bfloat162float(src[lane + 32 * i]);
-            ss = fmaf(e[i], e[i], ss);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = l2 ? 1.0f / sqrtf(ss + 1e-6f) : 1.0f;
-        float* dst = (m < M) ? kv[m] : qv;
-#pragma unroll
-        for (int i = 0; i < N / 32; ++i) dst[lane + 32 * i] = e[i] * inv;
-    }
-    for (int i = threadIdx.x; i < M * PB; i += blockDim.x) {
-        const int m = i / PB, j = i - m * PB;
-        vv[m][j] = __bfloat162float(xr[((int64_t)m * H + h) * P + p0 + j]);
-    }
-    if (threadIdx.x < M) gate_b[threadIdx.x] = write_gate(__bfloat162float(br[threadIdx.x * H + h]));
-    if (threadIdx.x == M)
-        gate_e = __double2float_rn(
-            exp((double)decay_gate(__bfloat162float(br[M * H + h]), dt_bias[h], A_log[h])));
-    __syncthreads();
-
-    // 3. the rule over the copies (decay on copy 0 only)
-    for (int m = 0; m < M; ++m) {
-        if (m == 0) {
-            const float e0 = gate_e;
-#pragma unroll
-            for (int rr = 0; rr < RPW; ++rr)
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) s[rr][c] *= e0;
-        }
-        float pp[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) pp[c] = 0.f;
-#pragma unroll
-        for (int rr = 0; rr < RPW; ++rr) {
-            const float kk = kv[m][warp * RPW + rr];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) pp[c] = fmaf(s[rr][c], kk, pp[c]);
-        }
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = pp[c];
-        __syncthreads();
-        if (threadIdx.x < PB) {
-            float d = 0.f;
-#pragma unroll
-            for (int w = 0; w < kDecWarps; ++w) d += red[w][threadIdx.x];
-            uu[threadIdx.x] = gate_b[m] * (vv[m][threadIdx.x] - d);
-        }
-        __syncthreads();
-        float u[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) u[c] = uu[lane * CPL + c];
-#pragma unroll
-        for (int rr = 0; rr < RPW; ++rr) {
-            const float kk = kv[m][warp * RPW + rr];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) s[rr][c] = fmaf(kk, u[c], s[rr][c]);
-        }
-    }
-
-    // 4. write the state back in place, then the output at the last copy
-#pragma unroll
-    for (int rr = 0; rr < RPW; ++rr) {
-        float* dst = st + (int64_t)(warp * RPW + rr) * P + lane * CPL;
-        if constexpr (CPL == 4) {
-            *reinterpret_cast<float4*>(dst) = make_float4(s[rr][0], s[rr][1], s[rr][2], s[rr][3]);
-        } else if constexpr (CPL == 2) {
-            *reinterpret_cast<float2*>(dst) = make_float2(s[rr][0], s[rr][1]);
-        } else {
-            dst[0] = s[rr][0];
-        }
-    }
-    {
-        float pp[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) pp[c] = 0.f;
-#pragma unroll
-        for (int rr = 0; rr < RPW; ++rr) {
-            const float qq = qv[warp * RPW + rr];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) pp[c] = fmaf(s[rr][c], qq, pp[c]);
-        }
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) red[warp][lane * CPL + c] = pp[c];
-        __syncthreads();
-        if (threadIdx.x < PB) {
-            float d = 0.f;
-#pragma unroll
-            for (int w = 0; w < kDecWarps; ++w) d += red[w][threadIdx.x];
-            o[(int64_t)rh * P + p0 + threadIdx.x] = __float2bfloat16_rn(scale * d);
-        }
-    }
-}
+// The decode step itself is in decode_step.cuh.
 
 }  // namespace gdn
 

@@ -359,7 +359,7 @@ gdn_status gdp_decode_step_indexed(const void* x, int64_t x_n_stride, const void
     if (!o || n_slots < 0 || (!state_idx && n_slots < n)) return GDN_ERR_INVALID_ARG;
     if (n_slots > 0 && (!state || !aligned16(state))) return GDN_ERR_INVALID_ARG;
     if (state_idx && (reinterpret_cast<uintptr_t>(state_idx) & 3u)) return GDN_ERR_INVALID_ARG;
-    if (M > gdn::kDecMaxM) return GDN_ERR_UNSUPPORTED;
+    if (M > gdn::dec::kMaxM) return GDN_ERR_UNSUPPORTED;
     if ((int64_t)n * H * 2 > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
     using bf = __nv_bfloat16;
     const int nb = n * H;
