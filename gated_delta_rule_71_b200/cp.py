@@ -9,7 +9,8 @@ Each rank holds one contiguous segment of the same sequences (dense batch,
 where (o_loc, h_loc) is the segment run from a zero state (rank 0: from the
 sequence's own h0) and M (key x key) is the segment's transition, the final
 state of a v = 0 run from h0 = I.  So every rank runs its segment and its
-transition locally, one all-gather exchanges (M_r, h_loc_r) -- key x key plus
+transition locally (one chunked call: the transition rides as extra heads),
+one all-gather exchanges (M_r, h_loc_r) -- key x key plus
 key x value fp32 per (sequence, head) -- and rank r forms its incoming state
 s_{r-1} with s_0 = h_loc_0, s_j = M_j s_{j-1} + h_loc_j, then adds the output
 of a v = 0 run from s_{r-1}.  The last rank's s is the sequences' final state.
@@ -51,12 +52,25 @@ def _lib_ops(scale: float) -> CpOps:
 
 def segment_local(q, k, v, g, beta, h0, ops: CpOps):
     """Phase 1 on one rank: (o_loc, h_loc, M) for its segment.  h0 is the
-    sequences' initial state on rank 0 and None elsewhere."""
+    sequences' initial state on rank 0 and None elsewhere.
+
+    With K == V the transition runs as H more heads of the same chunked call
+    (heads [H, 2H) see the segment's q, k, g, beta with v = 0 and start from
+    I): one launch with twice the (sequence, head) chains instead of two
+    launches, the same arithmetic per chain, so the same bits."""
     B, T, H, K = q.shape
+    V = v.shape[-1]
+    eye = torch.eye(K, dtype=torch.float32, device=q.device).expand(B, H, K, K)
+    if K == V:
+        h_start = h0 if h0 is not None else torch.zeros((B, H, K, V), dtype=torch.float32,
+                                                        device=q.device)
+        two = lambda t: torch.cat([t, t], dim=2)
+        o2, h2 = ops.chunk_fwd(two(q), two(k), torch.cat([v, torch.zeros_like(v)], dim=2),
+                               two(g), two(beta), torch.cat([h_start, eye], dim=1))
+        return o2[:, :, :H].contiguous(), h2[:, :H].contiguous(), h2[:, H:].contiguous()
     o_loc, h_loc = ops.chunk_fwd(q, k, v, g, beta, h0)
-    eye = torch.eye(K, dtype=torch.float32, device=q.device).expand(B, H, K, K).contiguous()
     zv = torch.zeros((B, T, H, K), dtype=v.dtype, device=v.device)
-    _, M = ops.chunk_fwd(q, k, zv, g, beta, eye)
+    _, M = ops.chunk_fwd(q, k, zv, g, beta, eye.contiguous())
     return o_loc, h_loc, M
 
 

@@ -67,3 +67,38 @@ def test_cp_emulated_ranks_match_one_pass(cuda_device, K, V, dtype, bounds, tol)
     assert relerr(o_cp.cpu(), ro) <= tol and relerr(h_cp.cpu(), rh) <= tol
     # and against the single pass itself (both sides on the same kernels)
     assert relerr(o_cp.cpu(), o1.double().cpu().numpy()) <= tol
+
+
+def test_cp_long_segments_match_the_oracle(cuda_device):
+    # three ranks' segments of 16K+ tokens each (ragged): the transition's
+    # product over a long segment runs through the bf16-operand tensor-core
+    # kernel from h0 = I, so its error is checked at length here
+    bounds = [0, 16384, 16384 + 16447, 16384 + 16447 + 16400]
+    w = I.small_chunk_workload(1, bounds[-1], 2, 128, 128, torch.bfloat16, h0=True, seed=75)
+    inp = I.chunk_inputs(w)
+    d = to_dev(inp, cuda_device)
+    beta, g = gdn.gate_prep(d["a"], d["b"], d["A_log"], d["dt_bias"])
+    o_cp, h_cp = _emulate(d["q"], d["k"], d["v"], g, beta, d["h0"], bounds, scale=1.0)
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    ro, rh = oracle.gdn_fwd(inp["q"], inp["k"], inp["v"], g.cpu(), beta.cpu(), h0=inp["h0"])
+    o_cp, h_cp = o_cp.cpu(), h_cp.cpu()
+    for r in range(3):
+        s = slice(bounds[r], bounds[r + 1])
+        assert relerr(o_cp[:, s], ro[:, s]) <= TOL_BF16, r
+    assert relerr(h_cp, rh) <= TOL_BF16
+
+
+def test_transition_rides_as_extra_heads_bit_for_bit(cuda_device):
+    # the stacked call (segment + transition as 2H heads) equals the two calls
+    w = I.small_chunk_workload(2, 300, 3, 128, 128, torch.bfloat16, h0=True, seed=76)
+    inp = I.chunk_inputs(w)
+    d = to_dev(inp, cuda_device)
+    beta, g = gdn.gate_prep(d["a"], d["b"], d["A_log"], d["dt_bias"])
+    ops = cp._lib_ops(1.0)
+    o_loc, h_loc, M = cp.segment_local(d["q"], d["k"], d["v"], g, beta, d["h0"], ops)
+    o1, h1 = gdn.chunk_fwd(d["q"], d["k"], d["v"], g, beta, h0=d["h0"])
+    eye = torch.eye(128, device=cuda_device).expand(2, 3, 128, 128).contiguous()
+    _, M1 = gdn.chunk_fwd(d["q"], d["k"], torch.zeros_like(d["v"]), g, beta, h0=eye)
+    torch.cuda.synchronize()
+    assert torch.equal(o_loc, o1) and torch.equal(h_loc, h1) and torch.equal(M, M1)
