@@ -14,25 +14,28 @@
 //   Ut^T = V^T Tb^T - S W^T                      ( = (U - W h)^T of the WY form)
 //   S'   = 2^G2_L S + (w Ut)^T K
 //   o_t  = scale (gam_t (S Q^T)_{:,t} + (Ut^T P^T)_{:,t})
-// Each (sequence, head) runs on a cluster of two CTAs, one per SM:
-//  * rank 0, "prep": three warpgroups, each owning every third chunk, its own
-//    K/Q stage and its own image buffer.  S_kk = [K; Q] K^T on tcgen05; the A
-//    and P rows from it; T by 16x16 blocks (substitution on the diagonal,
-//    warp-level tf32 MMAs off it).  The image [T' | Tb | P] (bf16) and the
-//    gate factors go to the chain CTA's slot with bulk copies that complete
-//    on the chain's mbarrier.  The K/Q stage is refilled as soon as S_kk has
-//    read it, so the next chunk's tiles load during this chunk's inverse.
-//  * rank 1, "chain": four warpgroups carry S in fp32 registers (value row =
+// Each (sequence, head) runs on a cluster of R + 1 CTAs, one per SM (R = 1, or
+// 2-3 when the chains leave SMs idle):
+//  * ranks 0..R-1, "prep": three warpgroups each; prep CTA r takes the chunks
+//    c with (c / 3) % R == r, its warpgroup j those with c % 3 == j, each
+//    warpgroup with its own K/Q stage and image buffer.  S_kk = [K; Q] K^T on
+//    tcgen05; the A and P rows from it; T by 16x16 blocks (substitution on the
+//    diagonal, warp-level tf32 MMAs off it).  The image [T' | Tb | P] (bf16)
+//    and the gate factors go to the chain CTA's slot c % 3 with bulk copies
+//    that complete on the chain's mbarrier.  The K/Q stage is refilled as soon
+//    as S_kk has read it, so the warpgroup's next chunk loads during this
+//    chunk's inverse.
+//  * rank R, "chain": four warpgroups carry S in fp32 registers (value row =
 //    tensor-memory lane, 32 key columns per warpgroup) and keep its bf16 copy
 //    in tensor memory, where it is the A operand of the chain's MMAs, so the
 //    serial part is two tcgen05 products per chunk (Ut^T, then dS) with no
 //    shared-memory round trip of the state.  W^T = K^T T'^T is formed on
-//    this SM one chunk ahead, from the K tile it loads anyway.  The output
-//    leaves tensor memory transposed (each warp writes 128 contiguous bytes
-//    per token) while the next chunk's Ut^T product runs.  A loader thread
-//    keeps K, V, Q tiles in flight (three, two and two buffers) and hands
-//    the slots back to the prep CTA; it never blocks on one resource while
-//    another is ready.
+//    this SM one chunk ahead, from the K tile it loads anyway.  The output is
+//    staged in a swizzled fp32 tile that a store warp writes with TMA while
+//    the next chunk runs.  A loader thread keeps K, V, Q tiles in flight
+//    (three, two and one buffers) and hands each slot back to the prep CTA
+//    that fills it next; it never blocks on one resource while another is
+//    ready.
 // Every wait is bounded: a wait that gives up sets the CTA's abort flag (later
 // waits fall through, so every barrier is still reached), records
 // GDN_ERR_TIMEOUT, and the issuing threads drain their copies and MMAs before
@@ -41,6 +44,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <mutex>
 #include <utility>
 
 #include "chunk_simt.cuh"
@@ -176,6 +180,7 @@ struct Params {
     float scale;
     void* o;
     float* hT;
+    int R;  // prep CTAs per cluster (ranks 0..R-1); the chain is rank R
 };
 
 // Bounded wait that honours the CTA's abort flag.  `cluster` selects acquire at
@@ -416,10 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
     volatile uint32_t* abort_flag = misc + 1;
 
     const uint32_t rank = tc::cluster_ctarank();
+    const uint32_t R = (uint32_t)p.R;  // prep CTAs of the cluster; the chain is rank R
+    const bool is_chain = rank == R;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = p.H;
     // the (sequence, head) of this cluster
-    const int sh = (int)(blockIdx.x >> 1);
+    const int sh = (int)(blockIdx.x / (R + 1u));
     const int head = sh % H;
     const int seq = p.order ? p.order[sh / H] : sh / H;
     int64_t cs, ce;
@@ -447,21 +454,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         // chain: arm the slot barriers for the first images before the prep CTA
         // can start a copy (it waits at the cluster barrier below)
-        if (rank == 1)
+        if (is_chain)
             for (int i = 0; i < NPREP; ++i) tc::mbar_arrive_expect_tx(&bars[C_TPF + i], kImgTx);
     }
-    const uint32_t ncols = rank == 0 ? P_TMEM_COLS : C_TMEM_COLS;
+    const uint32_t ncols = is_chain ? C_TMEM_COLS : P_TMEM_COLS;
     if (warp == 0) tc::tmem_alloc(&misc[0], ncols);
     tc::tc_before_sync();
     __syncthreads();
-    tc::cluster_sync();  // both CTAs' barriers initialised before any remote arrive
+    tc::cluster_sync();  // every CTA's barriers initialised before any remote arrive
     tc::tc_after_sync();
     // read through a warp reduction so the compiler treats it as warp-uniform (the
     // tcgen05 operands it feeds must be uniform)
     const uint32_t tmem = __reduce_max_sync(0xffffffffu, misc[0]);
 
-    if (rank == 0) {
+    if (!is_chain) {
         // ================================================================ prep
+        // prep CTA `rank` takes the chunks c with (c / NPREP) % R == rank; its
+        // warpgroup pg those with c % NPREP == pg, i.e. c = pg + NPREP (rank + R n)
         const int pg = warp >> 2;
         if (pg < NPREP) {
             const int pt = threadIdx.x - 128 * pg, pw = warp & 3;
@@ -479,9 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             uint64_t* sfree = &bars[P_FREE + pg];
             const uint32_t tcol = tmem + 64u * pg;
             // this warpgroup's slot in the chain CTA
-            const uint32_t r_sl = tc::mapa(sbase + C_OFF_SL + pg * SZ_TILES, 1);
-            const uint32_t r_sc0 = tc::mapa(sbase + C_OFF_SC, 1);  // gate-factor ring
-            const uint32_t r_tpf = tc::mapa(smem_u32(&bars[C_TPF + pg]), 1);
+            const uint32_t r_sl = tc::mapa(sbase + C_OFF_SL + pg * SZ_TILES, R);
+            const uint32_t r_sc0 = tc::mapa(sbase + C_OFF_SC, R);  // gate-factor ring
+            const uint32_t r_tpf = tc::mapa(smem_u32(&bars[C_TPF + pg]), R);
+            const int c0 = pg + NPREP * (int)rank, cstep = NPREP * (int)R;
             const uint32_t idS = tc::idesc_bf16(128, 64, 0, 0);
             auto issue_load = [&](int c) {
                 const int y = (int)(cs + (int64_t)C * c);
@@ -492,10 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 tc::tma_load_2d(kq_p + 24576, &p.tm_q, head * KD + 64, y, full);
             };
             int loads = 0;
-            if (pt == 0 && pg < nch) {
+            if (pt == 0 && c0 < nch) {
                 tc::prefetch_tmap(&p.tm_q);
                 tc::prefetch_tmap(&p.tm_k);
-                issue_load(pg);
+                issue_load(c0);
                 loads = 1;
             }
             int n = 0;
@@ -511,10 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 }
             };
             float gv_next, bv_next;
-            load_gb(pg, gv_next, bv_next);
-            for (int c = pg; c < nch; c += NPREP, ++n) {
+            load_gb(c0, gv_next, bv_next);
+            for (int c = c0; c < nch; c += cstep, ++n) {
                 const float gv = gv_next, bv = bv_next;
-                load_gb(c + NPREP, gv_next, bv_next);
+                load_gb(c + cstep, gv_next, bv_next);
                 wait(full, n & 1, abort_flag);
                 __syncwarp();
                 if (pw == 0) {
@@ -557,9 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 }
                 wait(mS, n & 1, abort_flag);
                 tc::tc_after_sync();
-                // the stage has been read by S_kk: the chunk after next may load into it
-                if (pt == 0 && c + NPREP < nch && !*abort_flag) {
-                    issue_load(c + NPREP);
+                // the stage has been read by S_kk: this warpgroup's next chunk may load into it
+                if (pt == 0 && c + cstep < nch && !*abort_flag) {
+                    issue_load(c + cstep);
                     ++loads;
                 }
                 tc::named_bar(bid, 128);  // gam / beta visible
@@ -638,8 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                 tc::fence_async_smem();
                 tc::named_bar(bid, 128);
                 if (pt == 0) {
-                    // ship the image once the chain has released the slot
-                    if (n >= 1) wait(sfree, (n - 1) & 1, abort_flag, true);
+                    // ship the image once the chain has released the slot (after its last
+                    // product of chunk c - NPREP; handed back to this warpgroup once per
+                    // job of it from chunk NPREP on)
+                    if (c >= NPREP) wait(sfree, (uint32_t)(n - (rank == 0 ? 1 : 0)) & 1u, abort_flag, true);
                     tc::bulk_s2cluster(r_sl, im, SZ_TILES, r_tpf);
                     tc::bulk_s2cluster(r_sc0 + (uint32_t)(c % NFAC) * kScalBytes, cst_u32, kScalBytes,
                                        r_tpf);
@@ -675,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
             if (lane == 0) {
                 // loader: K, V and Q tiles as their buffers fall free, and the slots
                 // back to the prep CTA once consumed; polls every resource in turn
-                const uint32_t r_free0 = tc::mapa(smem_u32(&bars[P_FREE]), 0);
+                const uint32_t l_free0 = smem_u32(&bars[P_FREE]);
                 tc::prefetch_tmap(&p.tm_k);
                 tc::prefetch_tmap(&p.tm_v);
                 tc::prefetch_tmap(&p.tm_q);
@@ -693,7 +705,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fwd_tc_kernel(const __grid_
                         // re-arm the slot's barrier for its next image, then hand it back
                         const int j = ns % NPREP;
                         tc::mbar_arrive_expect_tx(&bars[C_TPF + j], kImgTx);
-                        tc::mbar_arrive_cluster(r_free0 + 8 * j);
+                        // to the prep CTA that builds chunk ns + NPREP
+                        const uint32_t tr = (uint32_t)((ns + NPREP) / NPREP) % R;
+                        tc::mbar_arrive_cluster(tc::mapa(l_free0 + 8u * (uint32_t)j, tr));
                         ++ns;
                         prog = true;
                     }
@@ -1057,8 +1071,53 @@ inline bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t co
 
 }  // namespace tcf
 
-// Launches the kernel: one cluster of two CTAs per (sequence, head).  Returns
-// 0 on success, 1 when the tensor maps could not be built, 2 on a launch error.
+// Prep CTAs per cluster for `chains` clusters: 1, or 2-3 when the chains leave SMs
+// idle and every cluster of that size is resident at once (the chain then waits
+// less for its images).  The resident-cluster count is queried once per device,
+// output type and cluster size.
+template <class KernFn>
+inline int pick_prep_ctas(KernFn kern, bool obf16, int64_t chains) {
+    static std::mutex mu;
+    static int cache[64][2][4];  // [device][obf16][R]: resident clusters + 1 (0 = unknown)
+    int dev = 0, n_sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    if (cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 1;
+    for (int R = 3; R >= 2; --R) {
+        if (chains * (R + 1) > n_sms) continue;
+        int ncl;
+        {
+            std::lock_guard<std::mutex> lock(mu);
+            ncl = cache[dev][obf16][R] - 1;
+        }
+        if (ncl < 0) {
+            cudaLaunchConfig_t cfg;
+            memset(&cfg, 0, sizeof(cfg));
+            cfg.blockDim = dim3(tcf::kThreads, 1, 1);
+            cfg.dynamicSmemBytes = tcf::SMEM_BYTES;
+            cfg.gridDim = dim3((unsigned)(R + 1), 1, 1);
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)(R + 1);
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            ncl = 0;
+            if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess) {
+                (void)cudaGetLastError();
+                ncl = 0;
+            }
+            std::lock_guard<std::mutex> lock(mu);
+            cache[dev][obf16][R] = ncl + 1;
+        }
+        if (ncl >= chains) return R;
+    }
+    return 1;
+}
+
+// Launches the kernel: one cluster per (sequence, head), R prep CTAs and the
+// chain CTA.  Returns 0 on success, 1 when the tensor maps could not be built,
+// 2 on a launch error.
 inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cudaStream_t st) {
     tcf::Params p;
     memset(&p, 0, sizeof(p));
@@ -1084,15 +1143,17 @@ inline int launch_chunk_tc(const ChunkArgs& a, int64_t T_total, bool obf16, cuda
                              (int)tcf::SMEM_BYTES) != cudaSuccess)
         return 2;
     const int64_t chains = (int64_t)a.n_seq * a.H;
+    const int R = pick_prep_ctas(kern, obf16, chains);
+    p.R = R;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.blockDim = dim3(tcf::kThreads, 1, 1);
     cfg.dynamicSmemBytes = tcf::SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)(chains * 2), 1, 1);
+    cfg.gridDim = dim3((unsigned)(chains * (R + 1)), 1, 1);
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = (unsigned)(R + 1);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;

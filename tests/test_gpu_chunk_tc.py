@@ -7,6 +7,10 @@ one cluster of (prep, chain) CTAs per (sequence, head).
   tail chunks and bf16 output through direct stores: both paths in one call
   match the oracle.
 * The launch captures into a CUDA graph and replays to the same bits.
+* With few chains a cluster carries two or three prep CTAs (chunks dealt out by
+  (c / 3) % R): 2, 40 and 64 chains (three, two and one prep CTAs on a 148-SM
+  part) and a packed batch whose short sequences leave some prep CTAs idle
+  match the oracle.
 """
 import pytest
 import torch
@@ -90,3 +94,29 @@ def test_cuda_graph_capture_and_replay(cuda_device):
     torch.cuda.synchronize()
     assert gdn.device_status() == 0
     assert torch.equal(o, o_ref) and torch.equal(hT, h_ref)
+
+
+@pytest.mark.parametrize("B,H", [(1, 2), (5, 8), (4, 16)])
+def test_prep_ctas_per_cluster(cuda_device, B, H):
+    w = I.small_chunk_workload(B, 700, H, 128, 128, torch.bfloat16, h0=True, seed=340 + B)
+    inp, d, beta, g = _prep(w, cuda_device)
+    o, hT = gdn.chunk_fwd(d["q"], d["k"], d["v"], g, beta, h0=d["h0"])
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    ro, rh = oracle.gdn_fwd(inp["q"], inp["k"], inp["v"], g.cpu(), beta.cpu(), h0=inp["h0"])
+    assert relerr(o.cpu(), ro) <= TOL_BF16 and relerr(hT.cpu(), rh) <= TOL_BF16
+
+
+def test_prep_ctas_with_short_sequences(cuda_device):
+    # 1 to 13 chunks per sequence: with three prep CTAs, chunks 0-2 go to the
+    # first, 3-5 to the second, 6-8 to the third, 9-11 to the first again
+    lengths = [1, 64, 130, 250, 400, 577, 830]
+    w = I.small_chunk_workload(1, sum(lengths), 2, 128, 128, torch.bfloat16,
+                               n_seq_varlen=len(lengths), h0=True, seed=350)
+    inp, d, beta, g = _prep(w, cuda_device, lengths=lengths)
+    o, hT = gdn.chunk_fwd(d["q"], d["k"], d["v"], g, beta, h0=d["h0"], cu_seqlens=d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    ro, rh = oracle.gdn_fwd(inp["q"], inp["k"], inp["v"], g.cpu(), beta.cpu(), h0=inp["h0"],
+                            cu_seqlens=inp["cu_seqlens"])
+    assert relerr(o.cpu(), ro) <= TOL_BF16 and relerr(hT.cpu(), rh) <= TOL_BF16
