@@ -296,7 +296,8 @@ def test_decode_step_full_size_sampled(cuda_device, l2):
     assert relerr(st.cpu()[rows], rs) <= TOL_F32
 
 
-@pytest.mark.parametrize("N,P,M,H,G", [(64, 32, 1, 4, 2), (32, 128, 3, 6, 3), (128, 64, 8, 2, 1)])
+@pytest.mark.parametrize("N,P,M,H,G", [(64, 32, 1, 4, 2), (32, 128, 3, 6, 3), (128, 64, 8, 2, 1),
+                                       (128, 128, 3, 6, 2), (128, 128, 8, 4, 4), (128, 128, 1, 2, 1)])
 def test_decode_step_other_shapes(cuda_device, N, P, M, H, G):
     w = I.DecodeWorkload("custom", 9, M, H, G, P, N, seed=31)
     d = I.decode_inputs(w)
