@@ -84,7 +84,7 @@ __device__ __forceinline__ void conv_shift(const ConvIn& cv, const __nv_bfloat16
 }
 
 template <int N, int P, int PB, bool FUSED>
-__global__ void __launch_bounds__(256, (PB <= 64 ? (FUSED ? 3 : 4) : 2)) step_kernel(
+__global__ void __launch_bounds__(256, (PB <= 64 ? 4 : 2)) step_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t xs, const __nv_bfloat16* __restrict__ ba,
     int64_t bas, const float* __restrict__ A_log, const float* __restrict__ dt_bias, int M, int H,
     int G, float* __restrict__ state, const int32_t* __restrict__ state_idx, int n_slots,
@@ -117,22 +117,27 @@ __global__ void __launch_bounds__(256, (PB <= 64 ? (FUSED ? 3 : 4) : 2)) step_ke
         return;
     }
 
-    // 1. the state loads first (the only large traffic)
+    // 1. the state loads (the only large traffic): first thing in the plain form,
+    //    after the convolution in the fused form (so the convolution's registers
+    //    and the state's are not live together, and four blocks still fit per SM)
     float* st = state + ((int64_t)slot * H + h) * N * P + p0 + lane * CPL;
     float s[RPW][CPL];
+    auto load_state = [&]() {
 #pragma unroll
-    for (int rr = 0; rr < RPW; ++rr) {
-        const float* src = st + (int64_t)(warp * RPW + rr) * P;
-        if constexpr (CPL == 4) {
-            const float4 t = *reinterpret_cast<const float4*>(src);
-            s[rr][0] = t.x; s[rr][1] = t.y; s[rr][2] = t.z; s[rr][3] = t.w;
-        } else if constexpr (CPL == 2) {
-            const float2 t = *reinterpret_cast<const float2*>(src);
-            s[rr][0] = t.x; s[rr][1] = t.y;
-        } else {
-            s[rr][0] = src[0];
+        for (int rr = 0; rr < RPW; ++rr) {
+            const float* src = st + (int64_t)(warp * RPW + rr) * P;
+            if constexpr (CPL == 4) {
+                const float4 t = *reinterpret_cast<const float4*>(src);
+                s[rr][0] = t.x; s[rr][1] = t.y; s[rr][2] = t.z; s[rr][3] = t.w;
+            } else if constexpr (CPL == 2) {
+                const float2 t = *reinterpret_cast<const float2*>(src);
+                s[rr][0] = t.x; s[rr][1] = t.y;
+            } else {
+                s[rr][0] = src[0];
+            }
         }
-    }
+    };
+    if constexpr (!FUSED) load_state();
 
     // 2. the block's inputs: values of its slab, keys and query of its group
     //    (conv outputs in the fused form), normalised, and the gates
@@ -157,6 +162,7 @@ __global__ void __launch_bounds__(256, (PB <= 64 ? (FUSED ? 3 : 4) : 2)) step_ke
             vv[m][j] = chan(ch);
             conv_shift(cv, xr, slot, C, ch);  // this block's own channel
         }
+        load_state();
         __syncthreads();
     }
     for (int m = warp; m <= M; m += kWarps) {
