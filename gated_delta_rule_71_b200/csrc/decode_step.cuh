@@ -21,7 +21,10 @@
 // partials alternate between two buffers, so the next sum needs no second
 // barrier to protect this one's reads).
 // The state is read once and written once: 2*N*P*4 bytes per (request, head),
-// the HBM traffic that bounds the kernel.
+// the HBM traffic that bounds the kernel.  Both go with streaming cache hints
+// (evict first: the slab is touched once per step, so it should not push the rows
+// and gates out of L2), and the plain form keeps to 48 registers so that five
+// blocks, five 32 KB slabs, are in flight per SM.
 #pragma once
 
 #include "common.cuh"
@@ -84,7 +87,7 @@ __device__ __forceinline__ void conv_shift(const ConvIn& cv, const __nv_bfloat16
 }
 
 template <int N, int P, int PB, bool FUSED>
-__global__ void __launch_bounds__(256, (PB <= 64 ? 4 : 2)) step_kernel(
+__global__ void __launch_bounds__(256, (PB <= 64 ? (FUSED ? 4 : 5) : 2)) step_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t xs, const __nv_bfloat16* __restrict__ ba,
     int64_t bas, const float* __restrict__ A_log, const float* __restrict__ dt_bias, int M, int H,
     int G, float* __restrict__ state, const int32_t* __restrict__ state_idx, int n_slots,
@@ -130,7 +133,7 @@ __global__ void __launch_bounds__(256, (PB <= 64 ? 4 : 2)) step_kernel(
                 const float4 t = *reinterpret_cast<const float4*>(src);
                 s[rr][0] = t.x; s[rr][1] = t.y; s[rr][2] = t.z; s[rr][3] = t.w;
             } else if constexpr (CPL == 2) {
-                const float2 t = *reinterpret_cast<const float2*>(src);
+                const float2 t = __ldcs(reinterpret_cast<const float2*>(src));
                 s[rr][0] = t.x; s[rr][1] = t.y;
             } else {
                 s[rr][0] = src[0];
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(256, (PB <= 64 ? 4 : 2)) step_kernel(
         if constexpr (CPL == 4) {
             *reinterpret_cast<float4*>(dst) = make_float4(s[rr][0], s[rr][1], s[rr][2], s[rr][3]);
         } else if constexpr (CPL == 2) {
-            *reinterpret_cast<float2*>(dst) = make_float2(s[rr][0], s[rr][1]);
+            __stcs(reinterpret_cast<float2*>(dst), make_float2(s[rr][0], s[rr][1]));
         } else {
             dst[0] = s[rr][0];
         }
